@@ -1,0 +1,431 @@
+"""Benchmark of the FP8 (E4M3) 128x128 block-scaled GEMM on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl {dg,reference}]
+
+Default workload: dense C = A.B^T with M = N = K = 4096, A from N(0,1) with 1% of
+rows x50, B from N(0,0.02), 128x128 block scales, BF16 out.  One step is the whole
+hot path on one batch: the BF16 -> E4M3 block quantization of A (activation scales
+recomputed per call) followed by the block-scaled GEMM; B is quantized once up
+front (weights and their scales are cached).  Inputs are resident in HBM; L2 is
+flushed before every step (a 256 MB write outside the timed events) and each step
+is timed with CUDA events on the launching stream.
+
+`value` is 2*M*N*K per step over the mean step time (TFLOP/s, summed over ranks
+for N > 1: each rank runs an independent replica, weak scaling).  `roofline`
+reports the GEMM kernel alone against the FP8 dense peak (the measured BF16 cuBLAS
+peak x 2, the nominal FP8/BF16 ratio).  `e2e` repeats the step through the same
+C ABI with pinned host buffers: host->device copy of A, quantize, GEMM,
+device->host copy of C.  `cpu_baseline` times the CPU oracle on a bounded sample.
+
+--impl reference times the CPU oracle (the only other implementation of the
+method here) on the same workload and metric, one bounded sample per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+L2_FLUSH_BYTES = 256 << 20
+FP8_OVER_BF16 = 2.0  # nominal dense FP8 / BF16 tensor throughput ratio on B200
+
+# DRAM bytes per launch of the dominant kernel from an ncu capture, keyed by the
+# hash of the kernel source it was taken on (stale figures are reported as null).
+NCU_TRAFFIC = {}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("gemm_tile.cu", "dg_device.cuh", "gemm_skinny.cu", "quantize.cu"):
+        with open(os.path.join(ROOT, "fp8_block_scaled_scales_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------ workloads
+WORKLOADS = ("dense_4096_outliers", "dense_512", "dense_8192", "skinny_m1", "skinny_m16", "skinny_m64",
+             "skinny_m128", "moe_g8", "moe_g64_zipf")
+
+
+def make_workload(name):
+    from fp8_block_scaled_scales_b200 import inputs
+    if name == "dense_4096_outliers":
+        return inputs.dense_4096_outliers()
+    if name == "dense_512":
+        return inputs.dense_512()
+    if name == "dense_8192":
+        return inputs.dense_8192()
+    if name.startswith("skinny_m"):
+        return inputs.skinny(int(name[len("skinny_m"):]))
+    if name == "moe_g8":
+        return inputs.moe_g8()
+    if name == "moe_g64_zipf":
+        return inputs.moe_g64_zipf()
+    raise SystemExit(f"unknown workload {name}")
+
+
+def workload_facts(w):
+    """(flops per step on real tokens, algorithmic GEMM bytes, rows of A, config dict)."""
+    from fp8_block_scaled_scales_b200.inputs import Grouped
+    if isinstance(w, Grouped):
+        real = int(w.counts.sum())
+        flops = 2.0 * real * w.N * w.K
+        Mt = w.M_total
+        gemm_bytes = Mt * w.K + w.G * w.N * w.K + Mt * w.N * 2 + 4 * (Mt // 128 + w.G * (w.N // 128)) * (w.K // 128)
+        cfg = {"workload": w.name, "experts": w.G, "N": w.N, "K": w.K, "token_slots": real,
+               "padded_rows": Mt}
+        return flops, gemm_bytes, Mt, cfg
+    flops = 2.0 * w.M * w.N * w.K
+    kb = w.K // 128
+    gemm_bytes = w.M * w.K + w.N * w.K + w.M * w.N * 2 + 4 * kb * (-(-w.M // 128) + -(-w.N // 128))
+    cfg = {"workload": w.name, "M": w.M, "N": w.N, "K": w.K}
+    return flops, gemm_bytes, w.M, cfg
+
+
+# -------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        sm, smax, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+def oracle_sample(w, rows_sample: int, seed: int = 0):
+    """Time the CPU oracle on `rows_sample` rows of the workload (quantize those rows
+    of A, then the block-scaled GEMM of those rows against all of B).  Returns
+    (seconds, flops done, threads, description).  B's quantization is not timed
+    (cached weights), matching the GPU step."""
+    import oracle
+    from fp8_block_scaled_scales_b200 import inputs
+    from fp8_block_scaled_scales_b200.inputs import Grouped
+    if isinstance(w, Grouped):
+        qb = np.stack([oracle.quantize_blockwise(inputs.bf16_bits(w.B[g]))[0] for g in range(w.G)])
+        sb = np.stack([oracle.quantize_blockwise(inputs.bf16_bits(w.B[g]))[1] for g in range(w.G)])
+        real = np.flatnonzero(inputs.real_row_mask(w.counts, w.offsets))
+        rng = np.random.default_rng(seed)
+        blocks = np.unique(rng.choice(real, size=max(1, rows_sample // 128), replace=False) // 128)
+        rows = np.concatenate([np.arange(b * 128, b * 128 + 128) for b in blocks])
+        t0 = time.perf_counter()
+        qa = np.zeros((w.M_total, w.K), np.uint8)
+        sa = np.ones((w.M_total // 128, w.K // 128), np.float32)
+        for b in blocks:
+            q, s = oracle.quantize_blockwise(inputs.bf16_bits(w.A[b * 128:(b + 1) * 128]))
+            qa[b * 128:(b + 1) * 128] = q
+            sa[b] = s[0]
+        ref = oracle.grouped_gemm_ref(qa, sa, qb, sb, w.offsets, rows)
+        out = oracle.bf16_from_double(np.nan_to_num(ref))
+        dt = time.perf_counter() - t0
+        nreal = int(np.isin(rows, real).sum())
+        desc = f"{len(rows)} rows ({nreal} real) in {len(blocks)} 128-row blocks x all {w.N} columns, K={w.K}"
+        return dt, 2.0 * nreal * w.N * w.K, oracle.num_threads(), desc
+    qb, sb = oracle.quantize_blockwise(inputs.bf16_bits(w.B))
+    rows = min(rows_sample, w.M)
+    rows = max(rows, 1)
+    t0 = time.perf_counter()
+    qa, sa = oracle.quantize_blockwise(inputs.bf16_bits(w.A[:rows]))
+    ref = oracle.gemm_ref(qa, sa, qb, sb)
+    out = oracle.bf16_from_double(ref)
+    dt = time.perf_counter() - t0
+    del out
+    desc = f"{rows} of {w.M} rows of C (all {w.N} columns, K={w.K}), their A quantization included"
+    return dt, 2.0 * rows * w.N * w.K, oracle.num_threads(), desc
+
+
+def default_oracle_rows(w) -> int:
+    from fp8_block_scaled_scales_b200.inputs import Grouped
+    if isinstance(w, Grouped):
+        return 1024
+    per_row = w.N * w.K
+    return int(max(1, min(w.M, 2.0e10 // per_row)))
+
+
+# ------------------------------------------------------------------ dist
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# -------------------------------------------------------------- dg impl
+def run_dg(args):
+    from fp8_block_scaled_scales_b200 import binding
+    from fp8_block_scaled_scales_b200.inputs import Grouped
+
+    world, rank, local = dist_setup(args.gpus)
+    w = make_workload(args.workload)
+    flops, gemm_bytes, rows_a, cfg = workload_facts(w)
+    grouped = isinstance(w, Grouped)
+    skinny = (not grouped) and w.M <= 128
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+
+    A_host = w.A.contiguous()
+    A = A_host.to(dev)
+    B = w.B.reshape(-1, w.K).to(dev) if grouped else w.B.to(dev)
+    qb, sb = binding.quantize_blockwise(B)                    # cached weights
+    if grouped:
+        qb = qb.view(w.G, w.N, w.K)
+        sb = sb.view(w.G, w.N // 128, w.K // 128)
+        off = torch.from_numpy(w.offsets).to(dev)
+    qa = torch.empty((rows_a, w.K), dtype=torch.uint8, device=dev)
+    sa = torch.empty((-(-rows_a // 128), w.K // 128), dtype=torch.float32, device=dev)
+    C = torch.empty((rows_a, w.N), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def gemm():
+        if grouped:
+            binding.grouped_gemm_contiguous(qa, sa, qb, sb, off, C=C)
+        else:
+            binding.gemm_blockscaled(qa, sa, qb, sb, C=C)
+
+    def step(x):
+        binding.quantize_blockwise(x, q=qa, s=sa)
+        gemm()
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step(A)
+    torch.cuda.synchronize()
+    if binding.last_device_status() != 0:
+        raise SystemExit("device status not OK after warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        barrier(world)
+        for i in range(K):
+            flush.fill_(i)
+            ev[i][0].record(stream)
+            binding.quantize_blockwise(A, q=qa, s=sa)
+            ev[i][1].record(stream)
+            gemm()
+            ev[i][2].record(stream)
+        barrier(world)
+    step_ms = [ev[i][0].elapsed_time(ev[i][2]) for i in range(K)]
+    gemm_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+    quant_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
+    if binding.last_device_status() != 0:
+        raise SystemExit("device status not OK after the timed region")
+    ms_step = max_over_ranks(statistics.mean(step_ms), world)
+    ms_gemm = max_over_ranks(statistics.mean(gemm_ms), world)
+
+    # end to end through the C ABI: pinned host A in, pinned host C out, every step
+    A_pin = A_host.pin_memory()
+    C_pin = torch.empty((rows_a, w.N), dtype=torch.bfloat16).pin_memory()
+    A_stage = torch.empty_like(A)
+    e2e_steps = max(3, min(K, 20))
+    for _ in range(2):
+        A_stage.copy_(A_pin, non_blocking=True)
+        step(A_stage)
+        C_pin.copy_(C, non_blocking=True)
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        A_stage.copy_(A_pin, non_blocking=True)
+        step(A_stage)
+        C_pin.copy_(C, non_blocking=True)
+    e1.record(stream)
+    barrier(world)
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+
+    peaks = load_peaks()
+    if skinny:
+        metric, unit = "FP8 block-scaled GEMM HBM GB/s (skinny M) and % of B200 HBM roofline", "GB/s"
+        per_step = gemm_bytes
+        value = world * per_step / (ms_step * 1e-3) / 1e9
+        e2e_value = world * per_step / (ms_e2e * 1e-3) / 1e9
+        achieved = gemm_bytes / (ms_gemm * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4)}
+    else:
+        metric = "FP8 block-scaled GEMM TFLOPS (dense + MoE grouped) and % of B200 FP8 roofline"
+        unit = "TFLOP/s"
+        value = world * flops / (ms_step * 1e-3) / 1e12
+        e2e_value = world * flops / (ms_e2e * 1e-3) / 1e12
+        achieved = flops / (ms_gemm * 1e-3) / 1e12
+        peak = peaks["bf16_tflops"] * FP8_OVER_BF16
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4)}
+    roof["peak_source"] = (f"{peaks['source']}: bf16 cuBLAS burst {peaks['bf16_tflops']} TF/s x {FP8_OVER_BF16}"
+                           if roof["bound"] == "tensor" else f"{peaks['source']}: HBM copy {peaks['hbm_gbs']} GB/s")
+    roof["traffic"] = NCU_TRAFFIC.get((args.workload, kernel_source_hash()))
+    roof["kernel_ms"] = round(ms_gemm, 5)
+    roof["quantize_ms"] = round(max_over_ranks(statistics.mean(quant_ms), world), 5)
+
+    out = {"metric": metric, "value": round(value, 2), "unit": unit, "n_gpus": world, "steps": K,
+           "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 (fp32 accumulate, bf16 out)",
+           "data": "synthetic (seeded N(0,1)/N(0,0.02) BF16, quantized per 128x128 block)",
+           "config": dict(cfg, l2="flushed before every step (256 MB write outside the events)",
+                          step="quantize A (BF16->E4M3+scales) + block-scaled GEMM; B quantized once",
+                          parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
+           "roofline": roof,
+           "e2e": {"value": round(e2e_value, 2), "unit": unit,
+                   "h2d_bytes_per_step": int(A_host.numel() * 2), "d2h_bytes_per_step": int(C.numel() * 2)},
+           "gpu_launches": 2 * K}
+    cs = clocks.summary()
+    if cs is not None:
+        out["clocks"] = cs
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, fl, cores, desc = oracle_sample(w, args.oracle_rows or default_oracle_rows(w))
+        if unit == "GB/s":
+            v = (gemm_bytes * fl / flops) / dt / 1e9
+        else:
+            v = fl / dt / 1e12
+        out["cpu_baseline"] = {"value": round(v, 6), "unit": unit, "cores": cores, "kind": "oracle",
+                               "sample": desc, "seconds": round(dt, 3)}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------ reference arm
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = make_workload(args.workload)
+    flops, gemm_bytes, rows_a, cfg = workload_facts(w)
+    rows = args.oracle_rows or max(1, default_oracle_rows(w) // 4)
+    times = []
+    for i in range(args.warmup + args.steps):
+        dt, fl, cores, desc = oracle_sample(w, rows, seed=i)
+        if i >= args.warmup:
+            times.append((dt, fl))
+    dt = sum(t for t, _ in times)
+    fl = sum(f for _, f in times)
+    value = fl / dt / 1e12
+    unit = "TFLOP/s"
+    metric = "FP8 block-scaled GEMM TFLOPS (dense + MoE grouped) and % of B200 FP8 roofline"
+    out = {"impl": "reference", "metric": metric, "value": round(value, 6), "unit": unit, "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * dt / len(times), 3),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+           "dtype": "e4m3 codes, fp64 oracle arithmetic", "data": "synthetic",
+           "config": dict(cfg, step="CPU oracle on a bounded row sample of the workload"),
+           "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": cores, "kind": "oracle",
+                            "sample": desc},
+           "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="dense_4096_outliers", choices=WORKLOADS)
+    ap.add_argument("--impl", default="dg", choices=["dg", "reference"])
+    ap.add_argument("--oracle-rows", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_dg(args)
+
+
+if __name__ == "__main__":
+    main()

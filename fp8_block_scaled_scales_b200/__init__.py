@@ -1,0 +1,8 @@
+"""FP8 (E4M3) 128x128 block-scaled GEMM for B200 (sm_100a).
+
+The compute lives in libdg.so (hand-written CUDA kernels behind a C ABI,
+include/dg.h); this package is its Python binding plus the seeded input
+generators used by the tests and the benchmark.
+"""
+from .binding import (DGError, gemm_blockscaled, grouped_gemm_contiguous,  # noqa: F401
+                      last_device_status, quantize_blockwise, set_kernel_control, version)

@@ -1,0 +1,204 @@
+// C ABI of libdg.so: argument validation, device checks, tensor-map encoding,
+// kernel dispatch and the device status word.  See include/dg.h for the contract.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdlib.h>
+
+#include <mutex>
+
+#include "dg_device.cuh"
+#include "dg_internal.h"
+
+namespace dg {
+
+// The device status word: [0] status of the first failure since the last read,
+// [1] role, [2] block, [3] step.  One per device (a module global).
+__device__ int g_status[4];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+int *g_status_addr[kMaxDevices];
+bool g_dev_ready[kMaxDevices];
+std::mutex g_mu;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+dg_status_t load_encoder() {
+    if (g_encode) return DG_OK;
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return DG_ERR_CUDA;
+    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    return DG_OK;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+uint64_t g_timeout_ns = 2000000000ull;
+int g_debug_flags = 0;
+
+}  // namespace
+
+KernelControl kernel_control() {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    KernelControl c;
+    c.timeout_ns = g_timeout_ns;
+    c.debug_flags = g_debug_flags;
+    c.status = (dev >= 0 && dev < kMaxDevices) ? g_status_addr[dev] : nullptr;
+    return c;
+}
+
+dg_status_t current_device(DeviceInfo *info, int *device) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DG_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return DG_ERR_UNSUPPORTED_DEVICE;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_dev_ready[dev]) {
+        int major = 0, minor = 0, sms = 0, smem = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+            return DG_ERR_CUDA;
+        g_dev[dev].ok = (major == 10 && minor == 0);
+        g_dev[dev].num_sms = sms;
+        g_dev[dev].max_smem_optin = smem;
+        if (load_encoder() != DG_OK) return DG_ERR_CUDA;
+        void *addr = nullptr;
+        if (g_dev[dev].ok) {
+            if (cudaGetSymbolAddress(&addr, g_status) != cudaSuccess) return DG_ERR_CUDA;
+        }
+        g_status_addr[dev] = static_cast<int *>(addr);
+        g_dev_ready[dev] = true;
+    }
+    *info = g_dev[dev];
+    if (device) *device = dev;
+    return info->ok ? DG_OK : DG_ERR_UNSUPPORTED_DEVICE;
+}
+
+dg_status_t make_tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, int elem_bytes,
+                         uint64_t rows, uint64_t cols, uint32_t box_rows, uint32_t box_cols,
+                         CUtensorMapSwizzle swizzle) {
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * static_cast<uint64_t>(elem_bytes)};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t elem_strides[2] = {1, 1};
+    const CUresult r = g_encode(map, dtype, 2, const_cast<void *>(base), dims, strides, box, elem_strides,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
+}
+
+}  // namespace dg
+
+using namespace dg;
+
+extern "C" {
+
+int dg_version(void) { return 100; }
+
+const char *dg_status_string(dg_status_t s) {
+    switch (s) {
+        case DG_OK: return "DG_OK";
+        case DG_ERR_INVALID_ARG: return "DG_ERR_INVALID_ARG: null pointer or bad argument";
+        case DG_ERR_SHAPE: return "DG_ERR_SHAPE: size outside the shape contract";
+        case DG_ERR_ALIGNMENT: return "DG_ERR_ALIGNMENT: pointer not aligned as required";
+        case DG_ERR_UNSUPPORTED_DEVICE: return "DG_ERR_UNSUPPORTED_DEVICE: needs compute capability 10.0 (sm_100a)";
+        case DG_ERR_CUDA: return "DG_ERR_CUDA: a CUDA call failed";
+        case DG_ERR_TIMEOUT: return "DG_ERR_TIMEOUT: a device pipeline wait ran past its limit";
+    }
+    return "unknown dg_status_t";
+}
+
+dg_status_t dg_get_last_device_status(cudaStream_t stream) {
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return DG_ERR_CUDA;
+    int h[4] = {0, 0, 0, 0};
+    if (cudaMemcpyFromSymbol(h, g_status, sizeof(h)) != cudaSuccess) return DG_ERR_CUDA;
+    const int zero[4] = {0, 0, 0, 0};
+    if (cudaMemcpyToSymbol(g_status, zero, sizeof(zero)) != cudaSuccess) return DG_ERR_CUDA;
+    return static_cast<dg_status_t>(h[0]);
+}
+
+// Test hook (declared in the test-only section of include/dg.h): sets the time
+// limit of the kernels' bounded waits and the debug switches for later launches.
+void dg_test_set_kernel_control(uint64_t timeout_ns, int debug_flags) {
+    g_timeout_ns = timeout_ns ? timeout_ns : 2000000000ull;
+    g_debug_flags = debug_flags;
+}
+
+dg_status_t dg_quantize_blockwise(const void *X_bf16, int64_t rows, int64_t cols, uint8_t *Q, float *S,
+                                  cudaStream_t stream) {
+    if (rows < 0 || cols < 0 || cols % 16 != 0) return DG_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return DG_OK;
+    if (!X_bf16 || !Q || !S) return DG_ERR_INVALID_ARG;
+    if (!aligned(X_bf16, 16) || !aligned(Q, 16) || !aligned(S, 4)) return DG_ERR_ALIGNMENT;
+    DeviceInfo dev;
+    dg_status_t st = current_device(&dev, nullptr);
+    if (st != DG_OK) return st;
+    return launch_quantize(X_bf16, rows, cols, Q, S, dev, stream);
+}
+
+static dg_status_t check_gemm_common(const uint8_t *A, const float *sA, const uint8_t *B, const float *sB,
+                                     const void *C) {
+    if (!A || !sA || !B || !sB || !C) return DG_ERR_INVALID_ARG;
+    if (!aligned(A, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(sA, 4) || !aligned(sB, 4))
+        return DG_ERR_ALIGNMENT;
+    return DG_OK;
+}
+
+dg_status_t dg_fp8_gemm_blockscaled_select(const uint8_t *A, const float *sA, const uint8_t *B, const float *sB,
+                                           void *C_bf16, int64_t M, int64_t N, int64_t K, dg_kernel_t kernel,
+                                           cudaStream_t stream) {
+    if (M < 0 || N < 0 || K <= 0 || K % 128 != 0 || N % 16 != 0) return DG_ERR_SHAPE;
+    // TMA coordinates are 32-bit signed
+    if (M > 0x7FFFFFFFLL || N > 0x7FFFFFFFLL || K > 0x7FFFFFFFLL) return DG_ERR_SHAPE;
+    if (kernel != DG_KERNEL_AUTO && kernel != DG_KERNEL_TILE && kernel != DG_KERNEL_SKINNY)
+        return DG_ERR_INVALID_ARG;
+    if (kernel == DG_KERNEL_SKINNY && M > 128) return DG_ERR_SHAPE;
+    if (M == 0 || N == 0) return DG_OK;
+    dg_status_t st = check_gemm_common(A, sA, B, sB, C_bf16);
+    if (st != DG_OK) return st;
+    DeviceInfo dev;
+    st = current_device(&dev, nullptr);
+    if (st != DG_OK) return st;
+    GemmArgs a = {A, sA, B, sB, C_bf16, nullptr, M, N, K, 0};
+    const bool skinny = kernel == DG_KERNEL_SKINNY || (kernel == DG_KERNEL_AUTO && M <= 128);
+    if (skinny) return launch_skinny_gemm(a, dev, stream);
+    return launch_tile_gemm(a, false, dev, stream);
+}
+
+dg_status_t dg_fp8_gemm_blockscaled(const uint8_t *A, const float *sA, const uint8_t *B, const float *sB,
+                                    void *C_bf16, int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
+    return dg_fp8_gemm_blockscaled_select(A, sA, B, sB, C_bf16, M, N, K, DG_KERNEL_AUTO, stream);
+}
+
+dg_status_t dg_fp8_grouped_gemm_contiguous(const uint8_t *A, const float *sA, const uint8_t *B, const float *sB,
+                                           void *C_bf16, const int32_t *group_offsets, int64_t M_total_capacity,
+                                           int G, int64_t N, int64_t K, cudaStream_t stream) {
+    if (M_total_capacity < 0 || M_total_capacity % 128 != 0 || N < 0 || N % 128 != 0 || K <= 0 ||
+        K % 128 != 0 || G < 1 || G > 1024)
+        return DG_ERR_SHAPE;
+    if (M_total_capacity > 0x7FFFFFFFLL || static_cast<int64_t>(G) * N > 0x7FFFFFFFLL || K > 0x7FFFFFFFLL)
+        return DG_ERR_SHAPE;
+    if (M_total_capacity == 0 || N == 0) return DG_OK;
+    if (!group_offsets) return DG_ERR_INVALID_ARG;
+    if (!aligned(group_offsets, 4)) return DG_ERR_ALIGNMENT;
+    dg_status_t st = check_gemm_common(A, sA, B, sB, C_bf16);
+    if (st != DG_OK) return st;
+    DeviceInfo dev;
+    st = current_device(&dev, nullptr);
+    if (st != DG_OK) return st;
+    GemmArgs a = {A, sA, B, sB, C_bf16, group_offsets, M_total_capacity, N, K, G};
+    return launch_tile_gemm(a, true, dev, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,56 @@
+// Host-side internals shared by the translation units of libdg.so.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/dg.h"
+
+namespace dg {
+
+// Per-device facts the dispatch needs (filled once per device).
+struct DeviceInfo {
+    int ok;          // compute capability 10.0
+    int num_sms;
+    int max_smem_optin;
+};
+
+// Returns DG_OK and fills *info for the current device, or an error status.
+dg_status_t current_device(DeviceInfo *info, int *device);
+
+// Encodes a 2-D tiled tensor map (row-major [rows][cols] of elem_bytes each)
+// with a box of box_cols x box_rows and the given swizzle.
+dg_status_t make_tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, int elem_bytes,
+                         uint64_t rows, uint64_t cols, uint32_t box_rows, uint32_t box_cols,
+                         CUtensorMapSwizzle swizzle);
+
+// Time limit for every bounded wait inside the kernels, and test-only switches.
+struct KernelControl {
+    uint64_t timeout_ns;
+    int debug_flags;  // bit 0: the tile kernel's producer skips its first stage
+    int *status;      // device address of the status word on the current device
+};
+// Valid after current_device() succeeded on the calling thread's device.
+KernelControl kernel_control();
+
+// --- launchers (validated arguments only) ----------------------------------
+struct GemmArgs {
+    const uint8_t *A;
+    const float *sA;
+    const uint8_t *B;
+    const float *sB;
+    void *C;
+    const int32_t *offsets;  // grouped only
+    int64_t M;               // dense: M, grouped: M_total_capacity
+    int64_t N;
+    int64_t K;
+    int G;                   // grouped only
+};
+
+dg_status_t launch_tile_gemm(const GemmArgs &a, bool grouped, const DeviceInfo &dev, cudaStream_t stream);
+dg_status_t launch_skinny_gemm(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream);
+dg_status_t launch_quantize(const void *X, int64_t rows, int64_t cols, uint8_t *Q, float *S,
+                            const DeviceInfo &dev, cudaStream_t stream);
+
+}  // namespace dg

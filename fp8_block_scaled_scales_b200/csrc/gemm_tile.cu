@@ -1,0 +1,356 @@
+// Persistent, warp-specialised FP8 (E4M3) block-scaled GEMM tile kernel for
+// sm_100a, dense and MoE grouped-contiguous forms.
+//
+// Method (2kiu.com/news/5461879 §2.1, §3.3; demingchina.com/news/60142 §3.1):
+//   C[m][n] = bf16( sum_kb sA[m/128][kb] * sB[n/128][kb] * P_kb[m][n] ),
+//   P_kb[m][n] = sum over the 128-wide K block kb of A[m][k] * B[n][k].
+// The tensor cores produce each P_kb in FP32 in tensor memory; the epilogue warps
+// multiply it by the block-scale product and add it to an FP32 accumulator held in
+// registers ("segmented accumulation", 2kiu.com/news/5461879 §3.3), in ascending kb.
+//
+// Roles (one CTA per SM, 12 warps):
+//   warp 0      TMA producer: 128-K slabs of A (128 rows) and B (BN rows) into a
+//               STAGES-deep ring of 128-byte-swizzled shared-memory stages
+//               (demingchina.com/news/60142 §3.3 producer/consumer split, §4.2
+//               swizzle, §4.3 multi-stage ring).
+//   warp 1      MMA issuer: one thread issues four tcgen05.mma (K = 32 each) per
+//               slab into one of two TMEM partial buffers, then commits to the
+//               stage's "empty" barrier and the buffer's "full" barrier.
+//   warps 2-3   idle (they hand their registers to the epilogue).
+//   warps 4-11  epilogue: per kb, tcgen05.ld the partial, acc += s * P_kb; after
+//               the last kb, round to BF16, stage in swizzled shared memory and
+//               TMA-store.  Warp w reads TMEM lanes 32*(w%4).., columns half
+//               (w-4)/4 of the tile.
+// While the epilogue works on buffer b the MMA warp fills buffer b^1, so the
+// tensor cores run ahead by one K block; at a tile boundary they run into the
+// next tile while the epilogue writes the previous tile's output.
+//
+// Grouped form: m-blocks run over the padded concatenation of the experts' rows;
+// the expert of m-block i is the g with off[g] <= 128 i < off[g+1] (the pages'
+// "experts stored contiguously by expert id", nxmr.cn/news/132300 §2.2); B is
+// addressed as rows g*N + n of a [G*N][K] matrix.
+#include <cuda_bf16.h>
+
+#include "dg_device.cuh"
+#include "dg_internal.h"
+
+namespace dg {
+
+struct TileParams {
+    const float *sA;
+    const float *sB;
+    const int32_t *offsets;
+    int G;
+    int num_m_cap;    // m-blocks of the allocation (dense: ceil(M/128))
+    int num_n_tiles;  // ceil(N / BN)
+    int M;            // rows of A and C (dense: M, grouped: capacity)
+    int N;
+    int Nb;           // ceil(N / 128)
+    int Kb;           // K / 128
+    uint64_t timeout_ns;
+    int *status;  // device status word
+    int debug_flags;
+};
+
+constexpr int kTileThreads = 384;
+constexpr int kRasterM = 8;  // m-blocks per raster group (L2 reuse of B tiles)
+
+__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int &mb, int &nb) {
+    const int group = t / (kRasterM * num_n);
+    const int first_m = group * kRasterM;
+    const int gm = min(kRasterM, num_m - first_m);
+    const int local = t - group * kRasterM * num_n;
+    mb = first_m + local % gm;
+    nb = local / gm;
+}
+
+// Expert owning padded row `row` (off[g] <= row < off[g+1]); requires row < off[G].
+__device__ __forceinline__ int expert_of_row(const int32_t *off, int G, int row) {
+    int lo = 0, hi = G;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldg(off + mid) <= row) lo = mid; else hi = mid;
+    }
+    return lo;
+}
+
+template <int BN, int STAGES>
+struct TileSmem {
+    static constexpr uint32_t kABytes = 128 * 128;
+    static constexpr uint32_t kBBytes = BN * 128;
+    static constexpr uint32_t kCBoxBytes = 32 * 64 * 2;  // one 32-row x 64-column BF16 box
+    static constexpr uint32_t kOffA = 0;
+    static constexpr uint32_t kOffB = kOffA + STAGES * kABytes;
+    static constexpr uint32_t kOffC = kOffB + STAGES * kBBytes;
+    static constexpr uint32_t kOffBar = kOffC + 8 * kCBoxBytes;
+    static constexpr uint32_t kNumBars = 2 * STAGES + 4;
+    static constexpr uint32_t kOffMisc = kOffBar + 8 * kNumBars;
+    static constexpr uint32_t kBytes = kOffMisc + 16;
+    static constexpr uint32_t kDynamicBytes = kBytes + 1024;  // slack for 1024-byte alignment
+};
+
+template <int BN, bool GROUPED, int STAGES>
+__global__ void __launch_bounds__(kTileThreads, 1)
+    tile_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmC, const TileParams p) {
+    using L = TileSmem<BN, STAGES>;
+    constexpr int kColsPerWarp = BN / 2;
+    constexpr uint32_t kTmemCols = 2 * BN;
+    constexpr uint32_t kIdesc = idesc_e4m3_f32(128, BN);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
+    uint64_t *empty = full + STAGES;
+    uint64_t *tfull = empty + STAGES;
+    uint64_t *tempty = tfull + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
+
+    const int warp = static_cast<int>(threadIdx.x >> 5);
+    const int lane = lane_id();
+
+    if (warp == 0 && lane == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 8);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmC);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int num_m = GROUPED ? min(p.num_m_cap, __ldg(p.offsets + p.G) / 128) : p.num_m_cap;
+    const int num_tiles = num_m * p.num_n_tiles;
+    const int Kb = p.Kb;
+
+    if (warp < 4) {
+        regs_dealloc<56>();
+        if (warp == 0 && lane == 0) {
+            // ------------------------------------------------------------ producer
+            uint32_t issued = 0, parity_bits = 0;
+            int it = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+                int mb, nb;
+                tile_coords(t, num_m, p.num_n_tiles, mb, nb);
+                int b_row = nb * BN;
+                if (GROUPED) b_row += expert_of_row(p.offsets, p.G, mb * 128) * p.N;
+                for (int kb = 0; kb < Kb; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t u = static_cast<uint32_t>(it / STAGES);
+                    if (!mbar_wait(&empty[s], (u & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
+                        record_failure(p.status, kStatusTimeout, 0, it);
+                        *abort_flag = 1;
+                        ok = false;
+                        break;
+                    }
+                    if ((p.debug_flags & 1) && it == 0) continue;  // test hook: never fill stage 0
+                    mbar_arrive_expect_tx(&full[s], L::kABytes + L::kBBytes);
+                    tma_load_2d(smem + L::kOffA + s * L::kABytes, &tmA, &full[s], kb * 128, mb * 128);
+                    tma_load_2d(smem + L::kOffB + s * L::kBBytes, &tmB, &full[s], kb * 128, b_row);
+                    issued |= 1u << s;
+                    parity_bits = (parity_bits & ~(1u << s)) | ((u & 1u) << s);
+                }
+            }
+            // every load issued must land before the CTA may exit
+            const int never = 0;
+            for (int s = 0; s < STAGES; ++s)
+                if (issued & (1u << s))
+                    if (!mbar_wait(&full[s], (parity_bits >> s) & 1u, &never, p.timeout_ns))
+                        record_failure(p.status, kStatusTimeout, 0, -1 - s);
+        } else if (warp == 1 && lane == 0) {
+            // ----------------------------------------------------------------- MMA
+            int it = 0, kc = 0;
+            bool ok = true;
+            const uint32_t a0 = smem_u32(smem + L::kOffA);
+            const uint32_t b0 = smem_u32(smem + L::kOffB);
+            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+                for (int kb = 0; kb < Kb; ++kb, ++it, ++kc) {
+                    const int s = it % STAGES;
+                    const uint32_t u = static_cast<uint32_t>(it / STAGES);
+                    const int buf = kc & 1;
+                    const uint32_t v = static_cast<uint32_t>(kc >> 1);
+                    if (!mbar_wait(&tempty[buf], (v & 1u) ^ 1u, abort_flag, p.timeout_ns) ||
+                        !mbar_wait(&full[s], u & 1u, abort_flag, p.timeout_ns)) {
+                        record_failure(p.status, kStatusTimeout, 1, it);
+                        *abort_flag = 1;
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t adesc = sdesc_kmajor_sw128(a0 + s * L::kABytes);
+                    const uint64_t bdesc = sdesc_kmajor_sw128(b0 + s * L::kBBytes);
+                    const uint32_t d = tmem_base + static_cast<uint32_t>(buf * BN);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)  // 32 bytes of K per instruction = +2 in the address field
+                        umma_e4m3(d, adesc + 2u * k, bdesc + 2u * k, kIdesc, k > 0 ? 1u : 0u);
+                    umma_commit(&empty[s]);
+                    umma_commit(&tfull[buf]);
+                }
+            }
+            // the tensor memory may only be released once every MMA issued is done
+            if (kc > 0) {
+                const int never = 0;
+                const int last = kc - 1;
+                if (!mbar_wait(&tfull[last & 1], static_cast<uint32_t>(last >> 1) & 1u, &never, p.timeout_ns))
+                    record_failure(p.status, kStatusTimeout, 1, -1);
+            }
+        }
+    } else {
+        regs_alloc<224>();
+        // -------------------------------------------------------------- epilogue
+        const int ew = warp - 4;
+        const int quarter = warp & 3;
+        const int half = ew >> 2;
+        uint8_t *cstage = smem + L::kOffC + ew * L::kCBoxBytes;
+        float acc[kColsPerWarp];
+        int kc = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+            int mb, nb;
+            tile_coords(t, num_m, p.num_n_tiles, mb, nb);
+            const int col0 = nb * BN + half * kColsPerWarp;
+            const int nb128 = col0 / 128;
+            const bool n_valid = nb128 < p.Nb;
+            int sb_row = nb128;
+            if (GROUPED) sb_row += expert_of_row(p.offsets, p.G, mb * 128) * p.Nb;
+            const float *sa_ptr = p.sA + static_cast<int64_t>(mb) * Kb;
+            const float *sb_ptr = p.sB + static_cast<int64_t>(sb_row) * Kb;
+#pragma unroll
+            for (int i = 0; i < kColsPerWarp; ++i) acc[i] = 0.0f;
+            for (int kb = 0; kb < Kb; ++kb, ++kc) {
+                const int buf = kc & 1;
+                const uint32_t v = static_cast<uint32_t>(kc >> 1);
+                const float scale = n_valid ? __ldg(sa_ptr + kb) * __ldg(sb_ptr + kb) : 0.0f;
+                if (!mbar_wait(&tfull[buf], v & 1u, abort_flag, p.timeout_ns)) {
+                    record_failure(p.status, kStatusTimeout, 2, kc);
+                    *abort_flag = 1;
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                       static_cast<uint32_t>(buf * BN + half * kColsPerWarp);
+#pragma unroll
+                for (int c = 0; c < kColsPerWarp / 32; ++c) {
+                    float part[32];
+                    tmem_load32(taddr + c * 32, part);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) acc[c * 32 + i] = fmaf(scale, part[i], acc[c * 32 + i]);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[buf]);
+            }
+            if (!ok) break;
+            // BF16 output: rows mb*128 + 32*quarter + lane, columns col0 .. col0 + kColsPerWarp
+            const int row0 = mb * 128 + quarter * 32;
+#pragma unroll
+            for (int j = 0; j < kColsPerWarp / 64; ++j) {
+                if (lane == 0) bulk_wait_read0();  // the previous store has finished reading cstage
+                __syncwarp();
+                uint8_t *rowp = cstage + lane * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const float *x = acc + j * 64 + c * 8;
+                    uint4 w;
+                    w.x = pack_bf16x2(x[0], x[1]);
+                    w.y = pack_bf16x2(x[2], x[3]);
+                    w.z = pack_bf16x2(x[4], x[5]);
+                    w.w = pack_bf16x2(x[6], x[7]);
+                    *reinterpret_cast<uint4 *>(rowp + ((c ^ (lane & 7)) << 4)) = w;
+                }
+                fence_async_smem();
+                __syncwarp();
+                // a box that starts past the matrix edge is skipped, not clipped
+                if (lane == 0 && col0 + j * 64 < p.N && row0 < p.M) {
+                    tma_store_2d(&tmC, cstage, col0 + j * 64, row0);
+                    bulk_commit();
+                }
+            }
+        }
+        if (lane == 0) bulk_wait_all0();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+template <int BN, bool GROUPED, int STAGES>
+static dg_status_t launch_tile_impl(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream) {
+    using L = TileSmem<BN, STAGES>;
+    static_assert(L::kDynamicBytes <= 232448, "shared memory budget");
+    CUtensorMap tmA, tmB, tmC;
+    const uint64_t b_rows = GROUPED ? static_cast<uint64_t>(a.G) * a.N : static_cast<uint64_t>(a.N);
+    dg_status_t st;
+    st = make_tmap_2d(&tmA, a.A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.M, a.K, 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != DG_OK) return st;
+    st = make_tmap_2d(&tmB, a.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, b_rows, a.K, BN, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != DG_OK) return st;
+    st = make_tmap_2d(&tmC, a.C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.M, a.N, 32, 64,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != DG_OK) return st;
+
+    const KernelControl ctl = kernel_control();
+    TileParams p;
+    p.sA = a.sA;
+    p.sB = a.sB;
+    p.offsets = a.offsets;
+    p.G = a.G;
+    p.num_m_cap = static_cast<int>((a.M + 127) / 128);
+    p.num_n_tiles = static_cast<int>((a.N + BN - 1) / BN);
+    p.M = static_cast<int>(a.M);
+    p.N = static_cast<int>(a.N);
+    p.Nb = static_cast<int>((a.N + 127) / 128);
+    p.Kb = static_cast<int>(a.K / 128);
+    p.timeout_ns = ctl.timeout_ns;
+    p.status = ctl.status;
+    p.debug_flags = ctl.debug_flags;
+
+    auto kernel = tile_gemm_kernel<BN, GROUPED, STAGES>;
+    static thread_local int configured_device = -1;
+    int device = 0;
+    cudaGetDevice(&device);
+    if (configured_device != device) {
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(L::kDynamicBytes)) != cudaSuccess)
+            return DG_ERR_CUDA;
+        configured_device = device;
+    }
+    const int64_t tiles = static_cast<int64_t>(p.num_m_cap) * p.num_n_tiles;
+    const int grid = static_cast<int>(tiles < dev.num_sms ? tiles : dev.num_sms);
+    kernel<<<grid, kTileThreads, L::kDynamicBytes, stream>>>(tmA, tmB, tmC, p);
+    return cudaGetLastError() == cudaSuccess ? DG_OK : DG_ERR_CUDA;
+}
+
+dg_status_t launch_tile_gemm(const GemmArgs &a, bool grouped, const DeviceInfo &dev, cudaStream_t stream) {
+    // BN = 256 columns per tile unless the matrix is narrower (fewer idle columns).
+    const bool narrow = a.N <= 128;
+    if (grouped) {
+        return narrow ? launch_tile_impl<128, true, 6>(a, dev, stream) : launch_tile_impl<256, true, 4>(a, dev, stream);
+    }
+    return narrow ? launch_tile_impl<128, false, 6>(a, dev, stream) : launch_tile_impl<256, false, 4>(a, dev, stream);
+}
+
+}  // namespace dg

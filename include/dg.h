@@ -1,0 +1,160 @@
+/*
+ * dg.h -- C ABI of libdg.so, an sm_100a (B200) implementation of the FP8 (E4M3)
+ * GEMM with 128x128 block-wise scaling, C = A * B^T, FP32 accumulation with a
+ * per-K-block scale promotion, BF16 output, in a dense and an MoE
+ * grouped-contiguous form, plus the BF16 -> E4M3 block quantizer that makes its
+ * inputs.
+ *
+ * The method, as the DeepGEMM pages describe it:
+ *   - FP8 E4M3 inputs (1 sign, 4 exponent, 3 mantissa bits, largest value 448):
+ *     DeepGEMM FP8 write-up (demingchina.com/news/60142) §3.1 format table;
+ *     DeepGEMM library page (2kiu.com/news/5461879) §2.1.
+ *   - A and B cut into 128x128 blocks, one FP32 scale per block; each output
+ *     block's result is multiplied by the A-block and B-block scales:
+ *     2kiu.com/news/5461879 §2.1, §3.3 (FP32 scale storage).
+ *   - FP32 accumulation of FP8 products, long K accumulated in segments:
+ *     2kiu.com/news/5461879 §3.3.  Here every 128-wide K block's partial sum is
+ *     multiplied by sA[m/128][kb] * sB[n/128][kb] and added to an FP32 register
+ *     accumulator, in ascending kb order.
+ *   - Scales computed ahead of time and multiplied back at the output end:
+ *     demingchina.com/news/60142 §3.1.
+ *   - MoE experts stored contiguously by expert id as one long matrix, one
+ *     launch for all experts: nxmr.cn/news/132300 §2.2; expert N and K fixed by
+ *     the model, only the token count M varies: 2kiu.com/news/5461879 §2.2.
+ *
+ * Conventions for every entry point:
+ *   - All matrix pointers are DEVICE pointers owned by the caller.  The library
+ *     allocates nothing per call and never frees caller memory.
+ *   - Matrices are dense row-major.  FP8 data is raw E4M3 bytes; scales are FP32;
+ *     the output is BF16 (IEEE bfloat16 bit patterns).
+ *   - Every call is asynchronous and ordered on `stream` (0 = legacy default
+ *     stream).  Nothing synchronises the host.  Arguments are validated on the
+ *     host before anything is enqueued; on an error nothing is enqueued.
+ *   - A launch failure returns DG_ERR_CUDA.  Failures detected on the device
+ *     (a pipeline wait that exceeded its time limit) are recorded in a
+ *     per-process device status word; read it with dg_get_last_device_status().
+ *   - The device must be compute capability 10.0 (B200, sm_100a); otherwise
+ *     DG_ERR_UNSUPPORTED_DEVICE.  There is no fallback path.
+ *   - Calls that overlap on the GPU are independent unless they write the same
+ *     output.  Results are bitwise run-to-run deterministic.
+ */
+#ifndef DG_H_
+#define DG_H_
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DG_OK = 0,
+    DG_ERR_INVALID_ARG = 1,        /* null pointer where data is needed, bad enum */
+    DG_ERR_SHAPE = 2,              /* a size outside the shape contract below */
+    DG_ERR_ALIGNMENT = 3,          /* a pointer not aligned as required */
+    DG_ERR_UNSUPPORTED_DEVICE = 4, /* current device is not compute capability 10.0 */
+    DG_ERR_CUDA = 5,               /* a CUDA runtime/driver call failed */
+    DG_ERR_TIMEOUT = 6             /* device: a pipeline wait ran past its limit */
+} dg_status_t;
+
+/*
+ * BF16 -> E4M3 block quantizer (2kiu.com/news/5461879 §2.1 block-wise scaling,
+ * §3.3 FP32 scales; activation scales recomputed on every call, §4/§5).
+ *
+ * For each 128x128 block of X (edge blocks hold only the elements present):
+ *   amax = max |x|;  s = amax / 448 rounded to FP32 (s = 1 when amax == 0);
+ *   q = x / s rounded to FP32, then to the nearest E4M3 value (ties to the even
+ *       code, magnitudes above 448 saturate to 448, the sign of zero is kept).
+ *
+ * X_bf16 : [rows][cols] BF16, 16-byte aligned.
+ * Q      : [rows][cols] E4M3 bytes out, 16-byte aligned.
+ * S      : [ceil(rows/128)][ceil(cols/128)] FP32 out, 4-byte aligned.
+ * rows >= 0, cols >= 0, cols % 16 == 0.  rows == 0 or cols == 0 is a no-op.
+ * The result is bit-identical to the definition above.
+ */
+dg_status_t dg_quantize_blockwise(const void *X_bf16, int64_t rows, int64_t cols,
+                                  uint8_t *Q, float *S, cudaStream_t stream);
+
+/*
+ * Dense block-scaled GEMM, C = A * B^T (2kiu.com/news/5461879 §2.1, §3.3;
+ * demingchina.com/news/60142 §3.1, §3.3):
+ *   C[m][n] = bf16( sum_kb sA[m/128][kb] * sB[n/128][kb] *
+ *                   sum_{k in block kb} A[m][k] * B[n][k] )
+ *
+ * A  : [M][K] E4M3, 16-byte aligned.     sA : [ceil(M/128)][K/128] FP32.
+ * B  : [N][K] E4M3, 16-byte aligned.     sB : [ceil(N/128)][K/128] FP32.
+ * C  : [M][N] BF16 out, 16-byte aligned.
+ * M >= 0, N >= 0 with N % 16 == 0, K > 0 with K % 128 == 0.
+ * M == 0 or N == 0 is a no-op.  M <= 128 takes the skinny split-K kernel,
+ * larger M the persistent tile kernel; both compute the same formula.
+ */
+dg_status_t dg_fp8_gemm_blockscaled(const uint8_t *A, const float *sA,
+                                    const uint8_t *B, const float *sB, void *C_bf16,
+                                    int64_t M, int64_t N, int64_t K, cudaStream_t stream);
+
+/*
+ * MoE grouped-contiguous block-scaled GEMM (nxmr.cn/news/132300 §2.2;
+ * 2kiu.com/news/5461879 §2.2): expert g owns rows [off[g], off[g+1]) of A and
+ * C, every off[g] a multiple of 128, and for those rows
+ *   C[m][n] = bf16( sum_kb sA[m/128][kb] * sB[g][n/128][kb] *
+ *                   sum_k A[m][k] * B[g][n][k] ).
+ * Padding rows inside an expert's range are computed like real rows (zero rows
+ * of A give zero rows of C).  Rows at or beyond off[G] are not written.
+ *
+ * A  : [M_total_capacity][K] E4M3.        sA : [M_total_capacity/128][K/128] FP32.
+ * B  : [G][N][K] E4M3.                    sB : [G][N/128][K/128] FP32.
+ * C  : [M_total_capacity][N] BF16 out.
+ * group_offsets : DEVICE int32 [G+1], off[0] == 0, non-decreasing, each a
+ *                 multiple of 128, off[G] <= M_total_capacity.  Read on the
+ *                 device, so it may be produced by an earlier kernel on `stream`.
+ * M_total_capacity % 128 == 0, 1 <= G <= 1024, N % 128 == 0, K % 128 == 0, K > 0.
+ * M_total_capacity == 0 or N == 0 is a no-op.
+ */
+dg_status_t dg_fp8_grouped_gemm_contiguous(const uint8_t *A, const float *sA,
+                                           const uint8_t *B, const float *sB,
+                                           void *C_bf16, const int32_t *group_offsets,
+                                           int64_t M_total_capacity, int G,
+                                           int64_t N, int64_t K, cudaStream_t stream);
+
+/*
+ * Kernel selection for the dense GEMM, for tests and measurement.  AUTO is the
+ * dispatch dg_fp8_gemm_blockscaled uses.  TILE forces the persistent tile
+ * kernel; SKINNY forces the split-K kernel (M <= 128 only, else DG_ERR_SHAPE).
+ */
+typedef enum { DG_KERNEL_AUTO = 0, DG_KERNEL_TILE = 1, DG_KERNEL_SKINNY = 2 } dg_kernel_t;
+
+dg_status_t dg_fp8_gemm_blockscaled_select(const uint8_t *A, const float *sA,
+                                           const uint8_t *B, const float *sB, void *C_bf16,
+                                           int64_t M, int64_t N, int64_t K,
+                                           dg_kernel_t kernel, cudaStream_t stream);
+
+/* Human-readable name of a status code (static storage). */
+const char *dg_status_string(dg_status_t status);
+
+/*
+ * Synchronises `stream`, returns the device status word recorded by kernels of
+ * this library on the current device since the previous call (DG_OK if none),
+ * and clears it.
+ */
+dg_status_t dg_get_last_device_status(cudaStream_t stream);
+
+/* Library ABI version (major * 100 + minor). */
+int dg_version(void);
+
+/*
+ * Test-only control of the kernels' failure detection.  Every wait inside the
+ * kernels gives up after timeout_ns nanoseconds (0 restores the default of 2 s),
+ * records DG_ERR_TIMEOUT in the device status word and lets the kernel finish
+ * cleanly.  debug_flags bit 0 makes the tile kernel's TMA producer skip its first
+ * shared-memory stage, so that the MMA warp's wait runs out: it exercises the
+ * timeout path without faulting or hanging the GPU.  Applies to launches made
+ * after the call, process-wide; not for production use.
+ */
+void dg_test_set_kernel_control(uint64_t timeout_ns, int debug_flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DG_H_ */

@@ -1,0 +1,37 @@
+"""Shared helpers for the GPU parity tests: run the oracle on the same seeded
+inputs the CUDA path gets and compare element by element."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from fp8_block_scaled_scales_b200 import inputs
+
+
+def oracle_quant(x_bf16: torch.Tensor):
+    """Oracle quantization of a CPU BF16 tensor (2-D or 3-D, blocks per last two dims)."""
+    if x_bf16.dim() == 3:
+        qs, ss = zip(*(oracle.quantize_blockwise(inputs.bf16_bits(x_bf16[g])) for g in range(x_bf16.shape[0])))
+        return np.stack(qs), np.stack(ss)
+    return oracle.quantize_blockwise(inputs.bf16_bits(x_bf16))
+
+
+def dev(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def c_f64(c: torch.Tensor) -> np.ndarray:
+    return c.float().cpu().numpy().astype(np.float64)
+
+
+def check(c_rows: np.ndarray, ref: np.ndarray, rms: float, what: str):
+    ok, nbad, ratio = oracle.check_tolerance(c_rows, ref, rms)
+    assert ok, f"{what}: {nbad} of {ref.size} outside |c-ref| <= 1e-2|ref| + 1e-3 rms (worst ratio {ratio:.3g})"
+    return ratio
+
+
+def stratified_rms(ref_rows: np.ndarray, row_weights: np.ndarray) -> float:
+    """RMS over all rows of a matrix from a weighted sample of its rows."""
+    ms = np.mean(ref_rows * ref_rows, axis=1)
+    return float(np.sqrt(np.sum(ms * row_weights) / np.sum(row_weights)))

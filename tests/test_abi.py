@@ -1,0 +1,65 @@
+"""The C ABI: libdg.so builds, loads without a GPU, exports every symbol that
+include/dg.h declares, and rejects bad arguments on the host before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from fp8_block_scaled_scales_b200 import binding
+from fp8_block_scaled_scales_b200 import build as dgbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "dg.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dg_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    dgbuild.build()
+    return binding.lib()
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for f in ("dg_quantize_blockwise", "dg_fp8_gemm_blockscaled", "dg_fp8_grouped_gemm_contiguous"):
+        assert f in names
+    assert set(names) == set(binding.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert isinstance(getattr(lib, name), ctypes._CFuncPtr)
+
+
+def test_status_strings_and_version(lib):
+    assert lib.dg_version() == 100
+    for code, name in binding.STATUS_NAMES.items():
+        assert lib.dg_status_string(code).decode().startswith(name)
+
+
+def test_host_validation_without_device(lib):
+    null = ctypes.c_void_p(0)
+    # shape errors and no-ops are decided before any CUDA call
+    assert lib.dg_quantize_blockwise(null, 4, 17, null, null, null) == 2
+    assert lib.dg_quantize_blockwise(null, -1, 16, null, null, null) == 2
+    assert lib.dg_quantize_blockwise(null, 0, 16, null, null, null) == 0
+    assert lib.dg_fp8_gemm_blockscaled(null, null, null, null, null, 8, 16, 100, null) == 2  # K % 128
+    assert lib.dg_fp8_gemm_blockscaled(null, null, null, null, null, 8, 24, 128, null) == 2  # N % 16
+    assert lib.dg_fp8_gemm_blockscaled(null, null, null, null, null, 8, 16, 0, null) == 2    # K == 0
+    assert lib.dg_fp8_gemm_blockscaled(null, null, null, null, null, 0, 16, 128, null) == 0  # M == 0
+    assert lib.dg_fp8_gemm_blockscaled(null, null, null, null, null, 8, 16, 128, null) == 1  # null data
+    assert lib.dg_fp8_gemm_blockscaled_select(null, null, null, null, null, 200, 16, 128, 2, null) == 2
+    assert lib.dg_fp8_gemm_blockscaled_select(null, null, null, null, null, 20, 16, 128, 7, null) == 1
+    assert lib.dg_fp8_grouped_gemm_contiguous(null, null, null, null, null, null, 100, 2, 128, 128, null) == 2
+    assert lib.dg_fp8_grouped_gemm_contiguous(null, null, null, null, null, null, 128, 0, 128, 128, null) == 2
+    assert lib.dg_fp8_grouped_gemm_contiguous(null, null, null, null, null, null, 128, 2, 64, 128, null) == 2
+    assert lib.dg_fp8_grouped_gemm_contiguous(null, null, null, null, null, null, 0, 2, 128, 128, null) == 0
+    assert lib.dg_fp8_grouped_gemm_contiguous(null, null, null, null, null, null, 128, 2, 128, 128, null) == 1
+    odd = ctypes.c_void_p(0x1001)
+    assert lib.dg_fp8_gemm_blockscaled(odd, odd, odd, odd, odd, 8, 16, 128, null) == 3
