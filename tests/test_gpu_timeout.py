@@ -1,0 +1,34 @@
+"""Failure detection on the GPU without a fault: every pipeline wait in the kernels
+is bounded.  A test hook makes the tile kernel's TMA producer skip its first stage,
+so the MMA warp's wait for that stage can never succeed; the kernel must give up
+after the (shortened) time limit, record DG_ERR_TIMEOUT in the device status word,
+release its tensor memory and return, leaving the context usable."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fp8_block_scaled_scales_b200 import binding, inputs
+
+from parity import c_f64, check, dev, oracle_quant
+
+pytestmark = pytest.mark.gpu
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    d = inputs.dense_custom(256, 512, 512, seed=9500)
+    qa, sa = oracle_quant(d.A)
+    qb, sb = oracle_quant(d.B)
+    A, SA, B, SB = dev(qa), dev(sa), dev(qb), dev(sb)
+    assert binding.last_device_status() == 0
+    try:
+        binding.set_kernel_control(timeout_ns=50_000_000, debug_flags=1)
+        binding.gemm_blockscaled(A, SA, B, SB, kernel="tile")
+        status = binding.last_device_status()
+    finally:
+        binding.set_kernel_control(0, 0)
+    assert status == 6, f"expected DG_ERR_TIMEOUT, got {status}"
+    # the same context still computes correct results
+    c = c_f64(binding.gemm_blockscaled(A, SA, B, SB, kernel="tile"))
+    assert binding.last_device_status() == 0
+    check(c, oracle.gemm_ref(qa, sa, qb, sb), None, "after timeout")
