@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libdg.so")
 DG_OK = 0
 STATUS_NAMES = {0: "DG_OK", 1: "DG_ERR_INVALID_ARG", 2: "DG_ERR_SHAPE", 3: "DG_ERR_ALIGNMENT",
                 4: "DG_ERR_UNSUPPORTED_DEVICE", 5: "DG_ERR_CUDA", 6: "DG_ERR_TIMEOUT"}
-KERNELS = {"auto": 0, "tile": 1, "skinny": 2}
+KERNELS = {"auto": 0, "tile": 1, "skinny": 2, "pair": 3}
 
 # every symbol include/dg.h declares
 EXPORTS = ("dg_quantize_blockwise", "dg_fp8_gemm_blockscaled", "dg_fp8_grouped_gemm_contiguous",

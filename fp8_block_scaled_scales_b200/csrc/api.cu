@@ -161,7 +161,8 @@ dg_status_t dg_fp8_gemm_blockscaled_select(const uint8_t *A, const float *sA, co
     if (M < 0 || N < 0 || K <= 0 || K % 128 != 0 || N % 16 != 0) return DG_ERR_SHAPE;
     // TMA coordinates are 32-bit signed
     if (M > 0x7FFFFFFFLL || N > 0x7FFFFFFFLL || K > 0x7FFFFFFFLL) return DG_ERR_SHAPE;
-    if (kernel != DG_KERNEL_AUTO && kernel != DG_KERNEL_TILE && kernel != DG_KERNEL_SKINNY)
+    if (kernel != DG_KERNEL_AUTO && kernel != DG_KERNEL_TILE && kernel != DG_KERNEL_SKINNY &&
+        kernel != DG_KERNEL_PAIR)
         return DG_ERR_INVALID_ARG;
     if (kernel == DG_KERNEL_SKINNY && M > 128) return DG_ERR_SHAPE;
     if (M == 0 || N == 0) return DG_OK;
@@ -171,9 +172,10 @@ dg_status_t dg_fp8_gemm_blockscaled_select(const uint8_t *A, const float *sA, co
     st = current_device(&dev, nullptr);
     if (st != DG_OK) return st;
     GemmArgs a = {A, sA, B, sB, C_bf16, nullptr, M, N, K, 0};
-    const bool skinny = kernel == DG_KERNEL_SKINNY || (kernel == DG_KERNEL_AUTO && M <= 128);
-    if (skinny) return launch_skinny_gemm(a, dev, stream);
-    return launch_tile_gemm(a, false, dev, stream);
+    if (kernel == DG_KERNEL_AUTO) kernel = M <= 128 ? DG_KERNEL_SKINNY : DG_KERNEL_PAIR;
+    if (kernel == DG_KERNEL_SKINNY) return launch_skinny_gemm(a, dev, stream);
+    if (kernel == DG_KERNEL_TILE) return launch_tile_gemm(a, false, dev, stream);
+    return N <= 128 ? launch_pair_gemm_n128(a, dev, stream) : launch_pair_gemm(a, dev, stream);
 }
 
 dg_status_t dg_fp8_gemm_blockscaled(const uint8_t *A, const float *sA, const uint8_t *B, const float *sB,

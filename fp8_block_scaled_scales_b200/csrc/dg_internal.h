@@ -49,6 +49,8 @@ struct GemmArgs {
 };
 
 dg_status_t launch_tile_gemm(const GemmArgs &a, bool grouped, const DeviceInfo &dev, cudaStream_t stream);
+dg_status_t launch_pair_gemm(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream);
+dg_status_t launch_pair_gemm_n128(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream);
 dg_status_t launch_skinny_gemm(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream);
 dg_status_t launch_quantize(const void *X, int64_t rows, int64_t cols, uint8_t *Q, float *S,
                             const DeviceInfo &dev, cudaStream_t stream);

@@ -1,0 +1,369 @@
+// CTA-pair (cta_group::2) FP8 block-scaled GEMM tile kernel for sm_100a, dense form.
+//
+// Same method and roles as the single-CTA tile kernel (gemm_tile.cu): per 128-wide
+// K block the tensor cores produce P_kb in FP32 in tensor memory and the epilogue
+// warps promote it, acc += sA[m/128][kb] * sB[n/128][kb] * P_kb, in ascending kb
+// (2kiu.com/news/5461879 §2.1, §3.3).  What changes is the MMA shape: the two CTAs
+// of a cluster pair compute one 256 x BN output tile together.  Each CTA loads its
+// own 128 rows of A and its own half (BN/2 rows) of the B tile; the even CTA's MMA
+// warp issues tcgen05.mma.cta_group::2 with M = 256, which reads the A halves from
+// both CTAs' shared memory, shares the two B halves across the pair and writes
+// each CTA's 128 rows x BN columns into that CTA's tensor memory.
+//
+// Per CTA and K block this moves 16 KB of A plus BN/2 x 128 bytes of B through
+// shared memory instead of 16 KB + BN x 128 bytes, so the same shared memory holds
+// a deeper ring (6 stages of 32 KB for BN = 256), and every B tile is fetched from
+// L2 once per pair.  The pages' cluster sharing of B tiles between neighbouring
+// CTAs (demingchina.com/news/60142 §3.4) is done here by the pair MMA itself, with
+// no multicast copy.
+//
+// Synchronisation across the pair:
+//   full[s]    even CTA only: its producer posts the byte count of both CTAs' loads,
+//              both producers' TMA loads complete on it.
+//   empty[s]   in both CTAs: the MMA commit arrives on both (multicast commit).
+//   tfull[b]   in both CTAs: the MMA commit arrives on both.
+//   tempty[b]  even CTA only: all 16 epilogue warps of the pair arrive on it.
+// All waits are CTA-scope polls of the waiting CTA's own barrier; the peer's
+// remote arrivals carry cluster-scope release semantics.
+#include <cuda_bf16.h>
+
+#include "dg_device.cuh"
+#include "dg_internal.h"
+
+namespace dg {
+
+struct PairParams {
+    const float *sA;
+    const float *sB;
+    int num_m;        // m-blocks: ceil(M / 128)
+    int num_n_tiles;  // ceil(N / BN)
+    int M, N;
+    int Nb;           // ceil(N / 128)
+    int Kb;           // K / 128
+    uint64_t timeout_ns;
+    int *status;
+    int debug_flags;
+};
+
+constexpr int kPairThreads = 384;
+constexpr int kPairRegsLaunch = 168;
+constexpr int kPairRegsProducer = 40;
+constexpr int kPairRegsEpilogue = 232;
+static_assert(128 * kPairRegsProducer + 256 * kPairRegsEpilogue <= kPairThreads * kPairRegsLaunch,
+              "setmaxnreg split exceeds the registers the block is launched with");
+constexpr int kPairRasterM = 4;  // m-pairs per raster group
+
+__device__ __forceinline__ void pair_tile_coords(int t, int num_mp, int num_n, int &mp, int &nb) {
+    const int group = t / (kPairRasterM * num_n);
+    const int first = group * kPairRasterM;
+    const int gm = min(kPairRasterM, num_mp - first);
+    const int local = t - group * kPairRasterM * num_n;
+    mp = first + local % gm;
+    nb = local / gm;
+}
+
+template <int BN, int STAGES, int NBUF>
+struct PairSmem {
+    static constexpr uint32_t kABytes = 128 * 128;
+    static constexpr uint32_t kBBytes = (BN / 2) * 128;
+    static constexpr uint32_t kCBoxBytes = 32 * 64 * 2;
+    static constexpr uint32_t kOffA = 0;
+    static constexpr uint32_t kOffB = kOffA + STAGES * kABytes;
+    static constexpr uint32_t kOffC = kOffB + STAGES * kBBytes;
+    static constexpr uint32_t kOffBar = kOffC + 8 * kCBoxBytes;
+    static constexpr uint32_t kNumBars = 2 * STAGES + 2 * NBUF;
+    static constexpr uint32_t kOffMisc = kOffBar + 8 * kNumBars;
+    static constexpr uint32_t kBytes = kOffMisc + 16;
+    static constexpr uint32_t kDynamicBytes = kBytes + 1024;
+};
+
+// Give in-flight TMA loads time to land before a CTA that gave up leaves.
+__device__ __forceinline__ void settle_after_abort() {
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 50000ull) {
+    }
+}
+
+template <int BN, int STAGES, int NBUF>
+__global__ void __launch_bounds__(kPairThreads, 1)
+    pair_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmC, const PairParams p) {
+    using L = PairSmem<BN, STAGES, NBUF>;
+    constexpr int kColsPerWarp = BN / 2;
+    constexpr uint32_t kTmemCols = tmem_cols_for(NBUF * BN);
+    constexpr uint32_t kIdesc = idesc_e4m3_f32(256, BN);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
+    uint64_t *empty = full + STAGES;
+    uint64_t *tfull = empty + STAGES;
+    uint64_t *tempty = tfull + NBUF;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
+
+    const int warp = static_cast<int>(threadIdx.x >> 5);
+    const int lane = lane_id();
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int pair = static_cast<int>(blockIdx.x >> 1);
+    const int num_pairs = static_cast<int>(gridDim.x >> 1);
+
+    if (warp == 0 && lane == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < NBUF; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 16);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmC);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int num_mp = (p.num_m + 1) / 2;
+    const int num_tiles = num_mp * p.num_n_tiles;
+    const int Kb = p.Kb;
+
+    if (warp < 4) {
+        regs_dealloc<kPairRegsProducer>();
+        if (warp == 0 && lane == 0) {
+            // ---------------------------------------------- producer (both CTAs)
+            const uint32_t full0 = mapa_shared(smem_u32(&full[0]), 0);  // the even CTA's full[0]
+            int it = 0;
+            bool ok = true;
+            for (int t = pair; t < num_tiles && ok; t += num_pairs) {
+                int mp, nb;
+                pair_tile_coords(t, num_mp, p.num_n_tiles, mp, nb);
+                const int a_row = (2 * mp + static_cast<int>(rank)) * 128;
+                const int b_row = nb * BN + static_cast<int>(rank) * (BN / 2);
+                for (int kb = 0; kb < Kb; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t u = static_cast<uint32_t>(it / STAGES);
+                    if (!mbar_wait(&empty[s], (u & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
+                        record_failure(p.status, kStatusTimeout, 20 + static_cast<int>(rank), it);
+                        *abort_flag = 1;
+                        ok = false;
+                        break;
+                    }
+                    if ((p.debug_flags & 1) && it == 0 && leader) continue;  // test hook: stage 0 never posted
+                    if (leader) mbar_arrive_expect_tx(&full[s], 2 * (L::kABytes + L::kBBytes));
+                    tma_load_2d_pair(smem + L::kOffA + s * L::kABytes, &tmA, full0 + 8u * s, kb * 128, a_row);
+                    tma_load_2d_pair(smem + L::kOffB + s * L::kBBytes, &tmB, full0 + 8u * s, kb * 128, b_row);
+                }
+            }
+            if (!ok) settle_after_abort();
+        } else if (warp == 1 && lane == 0 && leader) {
+            // ---------------------------------------------- MMA (even CTA only)
+            int it = 0, kc = 0;
+            bool ok = true;
+            const uint32_t a0 = smem_u32(smem + L::kOffA);
+            const uint32_t b0 = smem_u32(smem + L::kOffB);
+            for (int t = pair; t < num_tiles && ok; t += num_pairs) {
+                for (int kb = 0; kb < Kb; ++kb, ++it, ++kc) {
+                    const int s = it % STAGES;
+                    const uint32_t u = static_cast<uint32_t>(it / STAGES);
+                    const int buf = kc % NBUF;
+                    const uint32_t v = static_cast<uint32_t>(kc / NBUF);
+                    if (!mbar_wait(&tempty[buf], (v & 1u) ^ 1u, abort_flag, p.timeout_ns) ||
+                        !mbar_wait(&full[s], u & 1u, abort_flag, p.timeout_ns)) {
+                        record_failure(p.status, kStatusTimeout, 22, it);
+                        *abort_flag = 1;
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t adesc = sdesc_kmajor_sw128(a0 + s * L::kABytes);
+                    const uint64_t bdesc = sdesc_kmajor_sw128(b0 + s * L::kBBytes);
+                    const uint32_t d = tmem_base + static_cast<uint32_t>(buf * BN);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        umma_e4m3_pair(d, adesc + 2u * k, bdesc + 2u * k, kIdesc, k > 0 ? 1u : 0u);
+                    umma_commit_pair(&empty[s], 0x3);
+                    umma_commit_pair(&tfull[buf], 0x3);
+                }
+            }
+            if (kc > 0) {
+                const int never = 0;
+                const int last = kc - 1;
+                if (!mbar_wait(&tfull[last % NBUF], static_cast<uint32_t>(last / NBUF) & 1u, &never, p.timeout_ns))
+                    record_failure(p.status, kStatusTimeout, 22, -1);
+            }
+        }
+    } else {
+        regs_alloc<kPairRegsEpilogue>();
+        // -------------------------------------------------- epilogue (both CTAs)
+        const int ew = warp - 4;
+        const int quarter = warp & 3;
+        const int half = ew >> 2;
+        uint8_t *cstage = smem + L::kOffC + ew * L::kCBoxBytes;
+        const uint32_t tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);  // the even CTA's tempty[0]
+        float2 acc[kColsPerWarp / 2];
+        int kc = 0;
+        bool ok = true;
+        for (int t = pair; t < num_tiles && ok; t += num_pairs) {
+            int mp, nb;
+            pair_tile_coords(t, num_mp, p.num_n_tiles, mp, nb);
+            const int mb = 2 * mp + static_cast<int>(rank);
+            const int col0 = nb * BN + half * kColsPerWarp;
+            const int nb128 = col0 / 128;
+            const bool valid = nb128 < p.Nb && mb < p.num_m;
+            ScaleStream scales;
+            scales.start(p.sA + static_cast<int64_t>(valid ? mb : 0) * Kb,
+                         p.sB + static_cast<int64_t>(valid ? nb128 : 0) * Kb, 0, valid ? Kb : 0);
+#pragma unroll
+            for (int i = 0; i < kColsPerWarp / 2; ++i) acc[i] = make_float2(0.0f, 0.0f);
+            for (int kb = 0; kb < Kb; ++kb, ++kc) {
+                const int buf = kc % NBUF;
+                const uint32_t v = static_cast<uint32_t>(kc / NBUF);
+                const float scale = scales.scale(kb, kb);
+                const float2 s2 = make_float2(scale, scale);
+                if (!mbar_wait(&tfull[buf], v & 1u, abort_flag, p.timeout_ns)) {
+                    record_failure(p.status, kStatusTimeout, 24 + static_cast<int>(rank), kc);
+                    *abort_flag = 1;
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                       static_cast<uint32_t>(buf * BN + half * kColsPerWarp);
+#pragma unroll
+                for (int c = 0; c < kColsPerWarp / 64; ++c) {
+                    float part[64];
+                    tmem_load64(taddr + c * 64, part);
+                    if (c == kColsPerWarp / 64 - 1) {
+                        // this CTA's columns of the buffer are in registers: release them
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_cluster(tempty0 + 8u * buf);
+                    }
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        acc[c * 32 + i] = __ffma2_rn(make_float2(part[2 * i], part[2 * i + 1]), s2, acc[c * 32 + i]);
+                }
+            }
+            if (!ok) break;
+            const int row0 = mb * 128 + quarter * 32;
+#pragma unroll
+            for (int j = 0; j < kColsPerWarp / 64; ++j) {
+                if (lane == 0) bulk_wait_read0();
+                __syncwarp();
+                uint8_t *rowp = cstage + lane * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const float2 *x = acc + j * 32 + c * 4;
+                    uint4 w;
+                    w.x = pack_bf16x2(x[0].x, x[0].y);
+                    w.y = pack_bf16x2(x[1].x, x[1].y);
+                    w.z = pack_bf16x2(x[2].x, x[2].y);
+                    w.w = pack_bf16x2(x[3].x, x[3].y);
+                    *reinterpret_cast<uint4 *>(rowp + ((c ^ (lane & 7)) << 4)) = w;
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0 && col0 + j * 64 < p.N && row0 < p.M) {
+                    tma_store_2d(&tmC, cstage, col0 + j * 64, row0);
+                    bulk_commit();
+                }
+            }
+        }
+        if (lane == 0) bulk_wait_all0();
+    }
+
+    // neither CTA may leave while the other can still signal its barriers or
+    // read its shared memory
+    tc_fence_before();
+    __syncwarp();
+    cluster_sync();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, kTmemCols);
+    }
+}
+
+template <int BN, int STAGES, int NBUF>
+static dg_status_t launch_pair_impl(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream) {
+    using L = PairSmem<BN, STAGES, NBUF>;
+    static_assert(L::kDynamicBytes <= 232448, "shared memory budget");
+    CUtensorMap tmA, tmB, tmC;
+    dg_status_t st;
+    st = make_tmap_2d(&tmA, a.A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.M, a.K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != DG_OK) return st;
+    st = make_tmap_2d(&tmB, a.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.N, a.K, BN / 2, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != DG_OK) return st;
+    st = make_tmap_2d(&tmC, a.C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.M, a.N, 32, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != DG_OK) return st;
+
+    const KernelControl ctl = kernel_control();
+    PairParams p;
+    p.sA = a.sA;
+    p.sB = a.sB;
+    p.num_m = static_cast<int>((a.M + 127) / 128);
+    p.num_n_tiles = static_cast<int>((a.N + BN - 1) / BN);
+    p.M = static_cast<int>(a.M);
+    p.N = static_cast<int>(a.N);
+    p.Nb = static_cast<int>((a.N + 127) / 128);
+    p.Kb = static_cast<int>(a.K / 128);
+    p.timeout_ns = ctl.timeout_ns;
+    p.status = ctl.status;
+    p.debug_flags = ctl.debug_flags;
+
+    auto kernel = pair_gemm_kernel<BN, STAGES, NBUF>;
+    static thread_local int configured_device = -1;
+    static thread_local int max_pairs = 0;
+    int device = 0;
+    cudaGetDevice(&device);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(kPairThreads, 1, 1);
+    cfg.dynamicSmemBytes = L::kDynamicBytes;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (configured_device != device) {
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(L::kDynamicBytes)) != cudaSuccess)
+            return DG_ERR_CUDA;
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return DG_ERR_CUDA;
+        if (128 * kPairRegsProducer + 256 * kPairRegsEpilogue > kPairThreads * fa.numRegs) return DG_ERR_CUDA;
+        cfg.gridDim = dim3(static_cast<unsigned>(dev.num_sms & ~1), 1, 1);
+        int clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg) != cudaSuccess || clusters < 1)
+            return DG_ERR_CUDA;
+        max_pairs = clusters;
+        configured_device = device;
+    }
+    const int64_t tiles = static_cast<int64_t>((p.num_m + 1) / 2) * p.num_n_tiles;
+    const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
+    if (cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, tmC, p) != cudaSuccess) return DG_ERR_CUDA;
+    return DG_OK;
+}
+
+dg_status_t launch_pair_gemm(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream) {
+    return launch_pair_impl<256, 6, 2>(a, dev, stream);
+}
+
+dg_status_t launch_pair_gemm_n128(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream) {
+    return launch_pair_impl<128, 8, 4>(a, dev, stream);
+}
+
+}  // namespace dg

@@ -201,13 +201,14 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
         float acc[MP];
 #pragma unroll
         for (int j = 0; j < MP; ++j) acc[j] = 0.0f;
-        const float *sb_ptr = p.sB + static_cast<int64_t>(nb) * p.Kb;
+        ScaleStream scales;
+        scales.start(p.sA, p.sB + static_cast<int64_t>(nb) * p.Kb, kb0, kb1);
         bool ok = true;
         for (int i = 0; i < nkb; ++i) {
             const int buf = i & 1;
             const uint32_t v = static_cast<uint32_t>(i >> 1);
             const int kb = kb0 + i;
-            const float scale = __ldg(p.sA + kb) * __ldg(sb_ptr + kb);
+            const float scale = scales.scale(kb, i);
             if (!mbar_wait(&tfull[buf], v & 1u, abort_flag, p.timeout_ns)) {
                 record_failure(p.status, kStatusTimeout, 12, i);
                 *abort_flag = 1;

@@ -8,7 +8,10 @@
 // multiply it by the block-scale product and add it to an FP32 accumulator held in
 // registers ("segmented accumulation", 2kiu.com/news/5461879 §3.3), in ascending kb.
 //
-// Roles (one CTA per SM, 12 warps):
+// Roles (one CTA per SM, 12 warps; warpgroup 0 gives registers to the two
+// epilogue warpgroups with setmaxnreg: 128 x 40 + 256 x 232 = 384 x 168, the
+// registers the block is launched with -- the split must not exceed them, or
+// setmaxnreg.inc would wait forever; the launcher checks the compiled count):
 //   warp 0      TMA producer: 128-K slabs of A (128 rows) and B (BN rows) into a
 //               STAGES-deep ring of 128-byte-swizzled shared-memory stages
 //               (demingchina.com/news/60142 §3.3 producer/consumer split, §4.2
@@ -16,11 +19,13 @@
 //   warp 1      MMA issuer: one thread issues four tcgen05.mma (K = 32 each) per
 //               slab into one of two TMEM partial buffers, then commits to the
 //               stage's "empty" barrier and the buffer's "full" barrier.
-//   warps 2-3   idle (they hand their registers to the epilogue).
-//   warps 4-11  epilogue: per kb, tcgen05.ld the partial, acc += s * P_kb; after
-//               the last kb, round to BF16, stage in swizzled shared memory and
-//               TMA-store.  Warp w reads TMEM lanes 32*(w%4).., columns half
-//               (w-4)/4 of the tile.
+//   warps 2-3   idle.
+//   warps 4-11  epilogue: per kb, tcgen05.ld the partial 64 columns at a time,
+//               release the TMEM buffer as soon as the last load has landed, and
+//               acc += s * P_kb with packed FP32 FMAs; after the last kb, round to
+//               BF16, stage in swizzled shared memory and TMA-store.  Warp w reads
+//               TMEM lanes 32*(w%4).. (the lane quarter its warp id allows) and
+//               columns half (w-4)/4 of the tile.
 // While the epilogue works on buffer b the MMA warp fills buffer b^1, so the
 // tensor cores run ahead by one K block; at a tile boundary they run into the
 // next tile while the epilogue writes the previous tile's output.
@@ -53,6 +58,11 @@ struct TileParams {
 };
 
 constexpr int kTileThreads = 384;
+constexpr int kRegsLaunch = 168;    // 65536 / 384 rounded down to a multiple of 8
+constexpr int kRegsProducer = 40;   // warpgroup 0 (TMA, MMA, two idle warps)
+constexpr int kRegsEpilogue = 232;  // warpgroups 1 and 2
+static_assert(128 * kRegsProducer + 256 * kRegsEpilogue <= kTileThreads * kRegsLaunch,
+              "setmaxnreg split exceeds the registers the block is launched with");
 constexpr int kRasterM = 8;  // m-blocks per raster group (L2 reuse of B tiles)
 
 __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int &mb, int &nb) {
@@ -74,7 +84,7 @@ __device__ __forceinline__ int expert_of_row(const int32_t *off, int G, int row)
     return lo;
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int NBUF>
 struct TileSmem {
     static constexpr uint32_t kABytes = 128 * 128;
     static constexpr uint32_t kBBytes = BN * 128;
@@ -83,19 +93,19 @@ struct TileSmem {
     static constexpr uint32_t kOffB = kOffA + STAGES * kABytes;
     static constexpr uint32_t kOffC = kOffB + STAGES * kBBytes;
     static constexpr uint32_t kOffBar = kOffC + 8 * kCBoxBytes;
-    static constexpr uint32_t kNumBars = 2 * STAGES + 4;
+    static constexpr uint32_t kNumBars = 2 * STAGES + 2 * NBUF;
     static constexpr uint32_t kOffMisc = kOffBar + 8 * kNumBars;
     static constexpr uint32_t kBytes = kOffMisc + 16;
     static constexpr uint32_t kDynamicBytes = kBytes + 1024;  // slack for 1024-byte alignment
 };
 
-template <int BN, bool GROUPED, int STAGES>
+template <int BN, bool GROUPED, int STAGES, int NBUF>
 __global__ void __launch_bounds__(kTileThreads, 1)
     tile_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, const TileParams p) {
-    using L = TileSmem<BN, STAGES>;
+    using L = TileSmem<BN, STAGES, NBUF>;
     constexpr int kColsPerWarp = BN / 2;
-    constexpr uint32_t kTmemCols = 2 * BN;
+    constexpr uint32_t kTmemCols = tmem_cols_for(NBUF * BN);
     constexpr uint32_t kIdesc = idesc_e4m3_f32(128, BN);
 
     extern __shared__ uint8_t smem_raw[];
@@ -103,7 +113,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
     uint64_t *empty = full + STAGES;
     uint64_t *tfull = empty + STAGES;
-    uint64_t *tempty = tfull + 2;
+    uint64_t *tempty = tfull + NBUF;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
 
@@ -115,7 +125,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < NBUF; ++b) {
             mbar_init(&tfull[b], 1);
             mbar_init(&tempty[b], 8);
         }
@@ -139,7 +149,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
     const int Kb = p.Kb;
 
     if (warp < 4) {
-        regs_dealloc<56>();
+        regs_dealloc<kRegsProducer>();
         if (warp == 0 && lane == 0) {
             // ------------------------------------------------------------ producer
             uint32_t issued = 0, parity_bits = 0;
@@ -183,8 +193,8 @@ __global__ void __launch_bounds__(kTileThreads, 1)
                 for (int kb = 0; kb < Kb; ++kb, ++it, ++kc) {
                     const int s = it % STAGES;
                     const uint32_t u = static_cast<uint32_t>(it / STAGES);
-                    const int buf = kc & 1;
-                    const uint32_t v = static_cast<uint32_t>(kc >> 1);
+                    const int buf = kc % NBUF;
+                    const uint32_t v = static_cast<uint32_t>(kc / NBUF);
                     if (!mbar_wait(&tempty[buf], (v & 1u) ^ 1u, abort_flag, p.timeout_ns) ||
                         !mbar_wait(&full[s], u & 1u, abort_flag, p.timeout_ns)) {
                         record_failure(p.status, kStatusTimeout, 1, it);
@@ -207,18 +217,18 @@ __global__ void __launch_bounds__(kTileThreads, 1)
             if (kc > 0) {
                 const int never = 0;
                 const int last = kc - 1;
-                if (!mbar_wait(&tfull[last & 1], static_cast<uint32_t>(last >> 1) & 1u, &never, p.timeout_ns))
+                if (!mbar_wait(&tfull[last % NBUF], static_cast<uint32_t>(last / NBUF) & 1u, &never, p.timeout_ns))
                     record_failure(p.status, kStatusTimeout, 1, -1);
             }
         }
     } else {
-        regs_alloc<224>();
+        regs_alloc<kRegsEpilogue>();
         // -------------------------------------------------------------- epilogue
         const int ew = warp - 4;
         const int quarter = warp & 3;
         const int half = ew >> 2;
         uint8_t *cstage = smem + L::kOffC + ew * L::kCBoxBytes;
-        float acc[kColsPerWarp];
+        float2 acc[kColsPerWarp / 2];
         int kc = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
@@ -229,14 +239,16 @@ __global__ void __launch_bounds__(kTileThreads, 1)
             const bool n_valid = nb128 < p.Nb;
             int sb_row = nb128;
             if (GROUPED) sb_row += expert_of_row(p.offsets, p.G, mb * 128) * p.Nb;
-            const float *sa_ptr = p.sA + static_cast<int64_t>(mb) * Kb;
-            const float *sb_ptr = p.sB + static_cast<int64_t>(sb_row) * Kb;
+            ScaleStream scales;
+            scales.start(p.sA + static_cast<int64_t>(mb) * Kb, p.sB + static_cast<int64_t>(sb_row) * Kb, 0,
+                         n_valid ? Kb : 0);
 #pragma unroll
-            for (int i = 0; i < kColsPerWarp; ++i) acc[i] = 0.0f;
+            for (int i = 0; i < kColsPerWarp / 2; ++i) acc[i] = make_float2(0.0f, 0.0f);
             for (int kb = 0; kb < Kb; ++kb, ++kc) {
-                const int buf = kc & 1;
-                const uint32_t v = static_cast<uint32_t>(kc >> 1);
-                const float scale = n_valid ? __ldg(sa_ptr + kb) * __ldg(sb_ptr + kb) : 0.0f;
+                const int buf = kc % NBUF;
+                const uint32_t v = static_cast<uint32_t>(kc / NBUF);
+                const float scale = scales.scale(kb, kb);
+                const float2 s2 = make_float2(scale, scale);
                 if (!mbar_wait(&tfull[buf], v & 1u, abort_flag, p.timeout_ns)) {
                     record_failure(p.status, kStatusTimeout, 2, kc);
                     *abort_flag = 1;
@@ -247,15 +259,19 @@ __global__ void __launch_bounds__(kTileThreads, 1)
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                        static_cast<uint32_t>(buf * BN + half * kColsPerWarp);
 #pragma unroll
-                for (int c = 0; c < kColsPerWarp / 32; ++c) {
-                    float part[32];
-                    tmem_load32(taddr + c * 32, part);
+                for (int c = 0; c < kColsPerWarp / 64; ++c) {
+                    float part[64];
+                    tmem_load64(taddr + c * 64, part);
+                    if (c == kColsPerWarp / 64 - 1) {
+                        // every column of this buffer is in registers: hand it back
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&tempty[buf]);
+                    }
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) acc[c * 32 + i] = fmaf(scale, part[i], acc[c * 32 + i]);
+                    for (int i = 0; i < 32; ++i)
+                        acc[c * 32 + i] = __ffma2_rn(make_float2(part[2 * i], part[2 * i + 1]), s2, acc[c * 32 + i]);
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&tempty[buf]);
             }
             if (!ok) break;
             // BF16 output: rows mb*128 + 32*quarter + lane, columns col0 .. col0 + kColsPerWarp
@@ -267,12 +283,12 @@ __global__ void __launch_bounds__(kTileThreads, 1)
                 uint8_t *rowp = cstage + lane * 128;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    const float *x = acc + j * 64 + c * 8;
+                    const float2 *x = acc + j * 32 + c * 4;
                     uint4 w;
-                    w.x = pack_bf16x2(x[0], x[1]);
-                    w.y = pack_bf16x2(x[2], x[3]);
-                    w.z = pack_bf16x2(x[4], x[5]);
-                    w.w = pack_bf16x2(x[6], x[7]);
+                    w.x = pack_bf16x2(x[0].x, x[0].y);
+                    w.y = pack_bf16x2(x[1].x, x[1].y);
+                    w.z = pack_bf16x2(x[2].x, x[2].y);
+                    w.w = pack_bf16x2(x[3].x, x[3].y);
                     *reinterpret_cast<uint4 *>(rowp + ((c ^ (lane & 7)) << 4)) = w;
                 }
                 fence_async_smem();
@@ -295,9 +311,9 @@ __global__ void __launch_bounds__(kTileThreads, 1)
     }
 }
 
-template <int BN, bool GROUPED, int STAGES>
+template <int BN, bool GROUPED, int STAGES, int NBUF>
 static dg_status_t launch_tile_impl(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream) {
-    using L = TileSmem<BN, STAGES>;
+    using L = TileSmem<BN, STAGES, NBUF>;
     static_assert(L::kDynamicBytes <= 232448, "shared memory budget");
     CUtensorMap tmA, tmB, tmC;
     const uint64_t b_rows = GROUPED ? static_cast<uint64_t>(a.G) * a.N : static_cast<uint64_t>(a.N);
@@ -328,7 +344,7 @@ static dg_status_t launch_tile_impl(const GemmArgs &a, const DeviceInfo &dev, cu
     p.status = ctl.status;
     p.debug_flags = ctl.debug_flags;
 
-    auto kernel = tile_gemm_kernel<BN, GROUPED, STAGES>;
+    auto kernel = tile_gemm_kernel<BN, GROUPED, STAGES, NBUF>;
     static thread_local int configured_device = -1;
     int device = 0;
     cudaGetDevice(&device);
@@ -336,6 +352,10 @@ static dg_status_t launch_tile_impl(const GemmArgs &a, const DeviceInfo &dev, cu
         if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(L::kDynamicBytes)) != cudaSuccess)
             return DG_ERR_CUDA;
+        // the register split inside the kernel must fit what a launch provides
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return DG_ERR_CUDA;
+        if (128 * kRegsProducer + 256 * kRegsEpilogue > kTileThreads * fa.numRegs) return DG_ERR_CUDA;
         configured_device = device;
     }
     const int64_t tiles = static_cast<int64_t>(p.num_m_cap) * p.num_n_tiles;
@@ -348,9 +368,9 @@ dg_status_t launch_tile_gemm(const GemmArgs &a, bool grouped, const DeviceInfo &
     // BN = 256 columns per tile unless the matrix is narrower (fewer idle columns).
     const bool narrow = a.N <= 128;
     if (grouped) {
-        return narrow ? launch_tile_impl<128, true, 6>(a, dev, stream) : launch_tile_impl<256, true, 4>(a, dev, stream);
+        return narrow ? launch_tile_impl<128, true, 6, 4>(a, dev, stream) : launch_tile_impl<256, true, 4, 2>(a, dev, stream);
     }
-    return narrow ? launch_tile_impl<128, false, 6>(a, dev, stream) : launch_tile_impl<256, false, 4>(a, dev, stream);
+    return narrow ? launch_tile_impl<128, false, 6, 4>(a, dev, stream) : launch_tile_impl<256, false, 4, 2>(a, dev, stream);
 }
 
 }  // namespace dg

@@ -32,22 +32,41 @@ constexpr int kQuantThreads = 256;
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// fl32(x / s) as far as its E4M3 rounding can tell (see the file comment).
-__device__ __forceinline__ float scaled(float x, float s, float r, bool fast_ok) {
-    float y = x * r;
-    const uint32_t bits = __float_as_uint(y);
-    const uint32_t mag = bits & 0x7FFFFFFFu;
-    const int d = static_cast<int>(bits & 0xFFFFFu) - 0x80000;
-    const bool near_mid = (d <= 6) && (d >= -6);
-    // below 2^-6 (biased exponent 121) E4M3 values are subnormal: other midpoints
-    if (!fast_ok || near_mid || mag < (121u << 23)) y = __fdiv_rn(x, s);
-    return y;
+// True when y = x * r might not round to the same E4M3 code as fl32(x / s): y is
+// within 6 FP32 ulps of an E4M3 rounding midpoint (bit 19 set, bits 0-18 clear,
+// i.e. bits[19:0] in [0x7FFFA, 0x80006]) or below 2^-6, where E4M3 is subnormal
+// and its midpoints sit at other bit positions.
+__device__ __forceinline__ bool needs_exact(float y) {
+    const uint32_t b = __float_as_uint(y);
+    const bool near_mid = ((b + 0x80006u) & 0xFFFFFu) <= 12u;
+    return near_mid || (fabsf(y) < 0x1p-6f);
 }
 
-__device__ __forceinline__ uint32_t to_e4m3x4(float a, float b, float c, float d) {
-    const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
-    const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+__device__ __forceinline__ uint32_t to_e4m3x4(float2 a, float2 b) {
+    const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(a, __NV_SATFINITE, __NV_E4M3);
+    const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(b, __NV_SATFINITE, __NV_E4M3);
     return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
+
+// Eight BF16 (one 16-byte group) -> eight E4M3 codes.
+__device__ __forceinline__ uint2 quantize8(uint4 v, float s, float2 r2, bool fast_ok) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float2 x[4], y[4];
+    bool slow = !fast_ok;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        x[j] = make_float2(bf16_lo(w[j]), bf16_hi(w[j]));
+        y[j] = __fmul2_rn(x[j], r2);
+        slow |= needs_exact(y[j].x) | needs_exact(y[j].y);
+    }
+    if (__builtin_expect(slow, 0)) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) y[j] = make_float2(__fdiv_rn(x[j].x, s), __fdiv_rn(x[j].y, s));
+    }
+    uint2 out;
+    out.x = to_e4m3x4(y[0], y[1]);
+    out.y = to_e4m3x4(y[2], y[3]);
+    return out;
 }
 
 __global__ void __launch_bounds__(kQuantThreads)
@@ -63,7 +82,7 @@ __global__ void __launch_bounds__(kQuantThreads)
     const bool col_ok = col < C;  // C % 16 == 0, so a group is whole or absent
 
     uint4 v[8];
-    uint32_t amax_bits = 0;
+    uint32_t m2 = 0;  // two 16-bit magnitude maxima side by side
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int64_t row = br * 128 + sub + 16 * i;
@@ -72,14 +91,16 @@ __global__ void __launch_bounds__(kQuantThreads)
         } else {
             v[i] = make_uint4(0, 0, 0, 0);
         }
-        // |x| ordering equals the ordering of (bits & 0x7fff) for non-NaN BF16
-        const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            amax_bits = max(amax_bits, w[j] & 0x7FFFu);
-            amax_bits = max(amax_bits, (w[j] >> 16) & 0x7FFFu);
-        }
     }
+    // |x| ordering equals the ordering of (bits & 0x7fff) for non-NaN BF16
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        m2 = __vmaxu2(m2, v[i].x & 0x7FFF7FFFu);
+        m2 = __vmaxu2(m2, v[i].y & 0x7FFF7FFFu);
+        m2 = __vmaxu2(m2, v[i].z & 0x7FFF7FFFu);
+        m2 = __vmaxu2(m2, v[i].w & 0x7FFF7FFFu);
+    }
+    uint32_t amax_bits = max(m2 & 0xFFFFu, m2 >> 16);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax_bits = max(amax_bits, __shfl_xor_sync(0xFFFFFFFFu, amax_bits, o));
     if ((tid & 31) == 0) red[tid >> 5] = amax_bits;
@@ -91,6 +112,7 @@ __global__ void __launch_bounds__(kQuantThreads)
     const float s = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
     const float r = __frcp_rn(s);
     const bool fast_ok = isfinite(r);
+    const float2 r2 = make_float2(r, r);
     if (tid == 0) S[br * Cb + bc] = s;
 
     if (!col_ok) return;
@@ -98,17 +120,7 @@ __global__ void __launch_bounds__(kQuantThreads)
     for (int i = 0; i < 8; ++i) {
         const int64_t row = br * 128 + sub + 16 * i;
         if (row >= R) break;
-        const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-        float f[8];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            f[2 * j] = scaled(bf16_lo(w[j]), s, r, fast_ok);
-            f[2 * j + 1] = scaled(bf16_hi(w[j]), s, r, fast_ok);
-        }
-        uint2 out;
-        out.x = to_e4m3x4(f[0], f[1], f[2], f[3]);
-        out.y = to_e4m3x4(f[4], f[5], f[6], f[7]);
-        *reinterpret_cast<uint2 *>(Q + row * C + col) = out;
+        *reinterpret_cast<uint2 *>(Q + row * C + col) = quantize8(v[i], s, r2, fast_ok);
     }
 }
 

@@ -87,7 +87,7 @@ dg_status_t dg_quantize_blockwise(const void *X_bf16, int64_t rows, int64_t cols
  * C  : [M][N] BF16 out, 16-byte aligned.
  * M >= 0, N >= 0 with N % 16 == 0, K > 0 with K % 128 == 0.
  * M == 0 or N == 0 is a no-op.  M <= 128 takes the skinny split-K kernel,
- * larger M the persistent tile kernel; both compute the same formula.
+ * larger M the persistent CTA-pair tile kernel; both compute the same formula.
  */
 dg_status_t dg_fp8_gemm_blockscaled(const uint8_t *A, const float *sA,
                                     const uint8_t *B, const float *sB, void *C_bf16,
@@ -119,10 +119,12 @@ dg_status_t dg_fp8_grouped_gemm_contiguous(const uint8_t *A, const float *sA,
 
 /*
  * Kernel selection for the dense GEMM, for tests and measurement.  AUTO is the
- * dispatch dg_fp8_gemm_blockscaled uses.  TILE forces the persistent tile
- * kernel; SKINNY forces the split-K kernel (M <= 128 only, else DG_ERR_SHAPE).
+ * dispatch dg_fp8_gemm_blockscaled uses: SKINNY for M <= 128, else PAIR.
+ *   TILE    persistent single-CTA kernel, 128 x 256 (128 x 128 if N <= 128) tiles;
+ *   SKINNY  split-K kernel for M <= 128 (larger M gives DG_ERR_SHAPE);
+ *   PAIR    persistent CTA-pair kernel, 256 x 256 (256 x 128 if N <= 128) tiles.
  */
-typedef enum { DG_KERNEL_AUTO = 0, DG_KERNEL_TILE = 1, DG_KERNEL_SKINNY = 2 } dg_kernel_t;
+typedef enum { DG_KERNEL_AUTO = 0, DG_KERNEL_TILE = 1, DG_KERNEL_SKINNY = 2, DG_KERNEL_PAIR = 3 } dg_kernel_t;
 
 dg_status_t dg_fp8_gemm_blockscaled_select(const uint8_t *A, const float *sA,
                                            const uint8_t *B, const float *sB, void *C_bf16,

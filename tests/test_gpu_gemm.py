@@ -33,12 +33,13 @@ SMALL = [(512, 512, 512), (256, 256, 128), (300, 272, 384), (129, 400, 256), (10
 
 
 @pytest.mark.parametrize("M,N,K", SMALL)
-def test_dense_tile_kernel_full_compare(M, N, K):
+@pytest.mark.parametrize("kernel", ["tile", "pair"])
+def test_dense_tile_kernels_full_compare(M, N, K, kernel):
     d = inputs.dense_custom(M, N, K, seed=8000 + M + N + K, std_b=0.5)
     qa, sa, qb, sb = quantized(d)
-    c = c_f64(run(qa, sa, qb, sb, kernel="tile"))
+    c = c_f64(run(qa, sa, qb, sb, kernel=kernel))
     ref = oracle.gemm_ref(qa, sa, qb, sb)
-    check(c, ref, None, f"tile {M}x{N}x{K}")
+    check(c, ref, None, f"{kernel} {M}x{N}x{K}")
 
 
 SKINNY = [(1, 16, 128), (1, 4096, 4096), (5, 272, 640), (16, 4096, 1024), (17, 512, 512),
@@ -46,8 +47,8 @@ SKINNY = [(1, 16, 128), (1, 4096, 4096), (5, 272, 640), (16, 4096, 1024), (17, 5
 
 
 @pytest.mark.parametrize("M,N,K", SKINNY)
-@pytest.mark.parametrize("kernel", ["skinny", "tile"])
-def test_dense_small_m_both_kernels(M, N, K, kernel):
+@pytest.mark.parametrize("kernel", ["skinny", "tile", "pair"])
+def test_dense_small_m_all_kernels(M, N, K, kernel):
     d = inputs.dense_custom(M, N, K, seed=8100 + M + N + K)
     qa, sa, qb, sb = quantized(d)
     c = c_f64(run(qa, sa, qb, sb, kernel=kernel))
@@ -75,7 +76,8 @@ def _exact_inputs(M, N, K, seed):
 
 
 @pytest.mark.parametrize("M,N,K,kernel", [(300, 400, 256, "tile"), (64, 272, 384, "skinny"),
-                                          (128, 256, 256, "tile"), (7, 4096, 256, "skinny")])
+                                          (128, 256, 256, "tile"), (7, 4096, 256, "skinny"),
+                                          (300, 400, 256, "pair"), (520, 128, 384, "pair")])
 def test_dense_exact_small_integers_bit_exact(M, N, K, kernel):
     """Integer E4M3 values and power-of-two scales: every step is exact, so the BF16
     output must equal the oracle's exactly."""
@@ -93,7 +95,7 @@ def test_dense_deterministic_and_no_stray_writes():
     qa, sa, qb, sb = quantized(d)
     A, SA, B, SB = dev(qa), dev(sa), dev(qb), dev(sb)
     guard = 4096
-    for kernel in ("tile",):
+    for kernel in ("tile", "pair"):
         buf = torch.full((M * N + 2 * guard,), -7.0, dtype=torch.bfloat16, device="cuda")
         c = buf[guard:guard + M * N].view(M, N)
         binding.gemm_blockscaled(A, SA, B, SB, C=c, kernel=kernel)
@@ -118,8 +120,9 @@ def test_dense_unit_scale_identity_invariant():
     sb = (2.0 ** rng.integers(-8, 8, size=(3, 3))).astype(np.float32)
     want = sb[np.arange(N)[None, :] // 128, np.arange(M)[:, None] // 128] * oracle.e4m3_decode(qb).T
     want = oracle.bf16_bits_to_double(oracle.bf16_from_double(want))
-    c = c_f64(run(qa, sa, qb, sb, kernel="tile"))
-    assert np.array_equal(c, want)
+    for kernel in ("tile", "pair"):
+        c = c_f64(run(qa, sa, qb, sb, kernel=kernel))
+        assert np.array_equal(c, want), kernel
 
 
 # ---------------------------------------------------------------- full-size workloads

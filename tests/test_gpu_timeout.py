@@ -15,7 +15,8 @@ from parity import c_f64, check, dev, oracle_quant
 pytestmark = pytest.mark.gpu
 
 
-def test_bounded_wait_reports_timeout_and_context_survives():
+@pytest.mark.parametrize("kernel", ["tile", "pair"])
+def test_bounded_wait_reports_timeout_and_context_survives(kernel):
     d = inputs.dense_custom(256, 512, 512, seed=9500)
     qa, sa = oracle_quant(d.A)
     qb, sb = oracle_quant(d.B)
@@ -23,12 +24,12 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     assert binding.last_device_status() == 0
     try:
         binding.set_kernel_control(timeout_ns=50_000_000, debug_flags=1)
-        binding.gemm_blockscaled(A, SA, B, SB, kernel="tile")
+        binding.gemm_blockscaled(A, SA, B, SB, kernel=kernel)
         status = binding.last_device_status()
     finally:
         binding.set_kernel_control(0, 0)
     assert status == 6, f"expected DG_ERR_TIMEOUT, got {status}"
     # the same context still computes correct results
-    c = c_f64(binding.gemm_blockscaled(A, SA, B, SB, kernel="tile"))
+    c = c_f64(binding.gemm_blockscaled(A, SA, B, SB, kernel=kernel))
     assert binding.last_device_status() == 0
     check(c, oracle.gemm_ref(qa, sa, qb, sb), None, "after timeout")
