@@ -217,6 +217,57 @@ __device__ __forceinline__ void tmem_load32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Issue a load of 32 consecutive FP32 columns of this warp's 32 TMEM lanes without
+// waiting.  The registers are written asynchronously: they may only be read after
+// tmem_wait32() on the same array, which ties them so that no use is hoisted above
+// the wait.
+__device__ __forceinline__ void tmem_load32_async(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+// 16-column variant of tmem_load32_async / tmem_wait32.
+__device__ __forceinline__ void tmem_load16_async(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait16(uint32_t (&r)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                   "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                   "+r"(r[14]), "+r"(r[15])
+                 :
+                 : "memory");
+}
+
+// Wait for every outstanding TMEM load of this thread; `r` (the most recent load's
+// destination) is tied through the wait.
+__device__ __forceinline__ void tmem_wait32(uint32_t (&r)[32]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                   "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                   "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]),
+                   "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]),
+                   "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+                 :
+                 : "memory");
+}
+
 // Load 64 consecutive FP32 columns of this warp's 32 TMEM lanes and wait.
 __device__ __forceinline__ void tmem_load64(uint32_t taddr, float (&v)[64]) {
     uint32_t r[64];
@@ -277,32 +328,29 @@ struct ScaleStream {
     const float *a;
     const float *b;
     int kb_end;
-    float a_cur, b_cur, a_next, b_next;
+    float cur, next;  // lane l: sA * sB of K block (chunk base + l)
 
-    __device__ __forceinline__ void load(int base, float &x, float &y) const {
-        const int k = base + lane_id_inline();
-        x = k < kb_end ? __ldg(a + k) : 0.0f;
-        y = k < kb_end ? __ldg(b + k) : 0.0f;
+    __device__ __forceinline__ float load(int base) const {
+        const int k = base + static_cast<int>(threadIdx.x & 31u);
+        return k < kb_end ? __ldg(a + k) * __ldg(b + k) : 0.0f;
     }
-    static __device__ __forceinline__ int lane_id_inline() { return static_cast<int>(threadIdx.x & 31u); }
 
-    // a, b point at K block 0 of the tile's sA and sB rows; K blocks [kb_begin, kb_end)
+    // a_row, b_row point at K block 0 of the tile's sA and sB rows; K blocks [kb_begin, end)
     __device__ __forceinline__ void start(const float *a_row, const float *b_row, int kb_begin, int end) {
         a = a_row;
         b = b_row;
         kb_end = end;
-        load(kb_begin, a_cur, b_cur);
-        load(kb_begin + 32, a_next, b_next);
+        cur = load(kb_begin);
+        next = load(kb_begin + 32);
     }
-    // product of the two block scales of K block kb; `i` = kb - kb_begin.  Called
-    // by all 32 lanes in order i = 0, 1, 2, ...
+    // block-scale product of K block kb; `i` = kb - kb_begin.  Called by all 32
+    // lanes in order i = 0, 1, 2, ...
     __device__ __forceinline__ float scale(int kb, int i) {
         if ((i & 31) == 0 && i > 0) {
-            a_cur = a_next;
-            b_cur = b_next;
-            load(kb + 32, a_next, b_next);
+            cur = next;
+            next = load(kb + 32);
         }
-        return __shfl_sync(0xFFFFFFFFu, a_cur, i & 31) * __shfl_sync(0xFFFFFFFFu, b_cur, i & 31);
+        return __shfl_sync(0xFFFFFFFFu, cur, i & 31);
     }
 };
 

@@ -20,8 +20,10 @@
 // Synchronisation across the pair:
 //   full[s]    even CTA only: its producer posts the byte count of both CTAs' loads,
 //              both producers' TMA loads complete on it.
-//   empty[s]   in both CTAs: the MMA commit arrives on both (multicast commit).
-//   tfull[b]   in both CTAs: the MMA commit arrives on both.
+//   empty[s]   in both CTAs: each CTA's epilogue arrives once it has seen tfull for
+//              the K block that used the stage (the pair's MMAs are then done).
+//   tfull[b]   in both CTAs: the MMA commit (multicast) arrives on both.
+// Two threads of the even CTA issue the MMAs, alternating K blocks.
 //   tempty[b]  even CTA only: all 16 epilogue warps of the pair arrive on it.
 // All waits are CTA-scope polls of the waiting CTA's own barrier; the peer's
 // remote arrivals carry cluster-scope release semantics.
@@ -47,9 +49,10 @@ struct PairParams {
 
 constexpr int kPairThreads = 384;
 constexpr int kPairRegsLaunch = 168;
-constexpr int kPairRegsProducer = 40;
-constexpr int kPairRegsEpilogue = 232;
-static_assert(128 * kPairRegsProducer + 256 * kPairRegsEpilogue <= kPairThreads * kPairRegsLaunch,
+template <int BN> __host__ __device__ constexpr int pair_regs_producer() { return BN == 256 ? 56 : 64; }
+template <int BN> __host__ __device__ constexpr int pair_regs_epilogue() { return BN == 256 ? 224 : 216; }
+static_assert(128 * pair_regs_producer<256>() + 256 * pair_regs_epilogue<256>() <= kPairThreads * kPairRegsLaunch &&
+                  128 * pair_regs_producer<128>() + 256 * pair_regs_epilogue<128>() <= kPairThreads * kPairRegsLaunch,
               "setmaxnreg split exceeds the registers the block is launched with");
 constexpr int kPairRasterM = 4;  // m-pairs per raster group
 
@@ -71,7 +74,7 @@ struct PairSmem {
     static constexpr uint32_t kOffB = kOffA + STAGES * kABytes;
     static constexpr uint32_t kOffC = kOffB + STAGES * kBBytes;
     static constexpr uint32_t kOffBar = kOffC + 8 * kCBoxBytes;
-    static constexpr uint32_t kNumBars = 2 * STAGES + 2 * NBUF;
+    static constexpr uint32_t kNumBars = 2 * STAGES + 2 * NBUF + 2;
     static constexpr uint32_t kOffMisc = kOffBar + 8 * kNumBars;
     static constexpr uint32_t kBytes = kOffMisc + 16;
     static constexpr uint32_t kDynamicBytes = kBytes + 1024;
@@ -89,7 +92,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     pair_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, const PairParams p) {
     using L = PairSmem<BN, STAGES, NBUF>;
-    constexpr int kColsPerWarp = BN / 2;
+        constexpr int kColsPerWarp = BN / 2;
     constexpr uint32_t kTmemCols = tmem_cols_for(NBUF * BN);
     constexpr uint32_t kIdesc = idesc_e4m3_f32(256, BN);
 
@@ -99,6 +102,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     uint64_t *empty = full + STAGES;
     uint64_t *tfull = empty + STAGES;
     uint64_t *tempty = tfull + NBUF;
+    uint64_t *mdone = tempty + NBUF;  // one per MMA thread: all its MMAs complete
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
 
@@ -114,6 +118,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
+        for (int q = 0; q < 2; ++q) mbar_init(&mdone[q], 1);
         for (int b = 0; b < NBUF; ++b) {
             mbar_init(&tfull[b], 1);
             mbar_init(&tempty[b], 16);
@@ -138,7 +143,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const int Kb = p.Kb;
 
     if (warp < 4) {
-        regs_dealloc<kPairRegsProducer>();
+        regs_dealloc<pair_regs_producer<BN>()>();
         if (warp == 0 && lane == 0) {
             // ---------------------------------------------- producer (both CTAs)
             const uint32_t full0 = mapa_shared(smem_u32(&full[0]), 0);  // the even CTA's full[0]
@@ -165,45 +170,47 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                 }
             }
             if (!ok) settle_after_abort();
-        } else if (warp == 1 && lane == 0 && leader) {
-            // ---------------------------------------------- MMA (even CTA only)
-            int it = 0, kc = 0;
-            bool ok = true;
+        } else if ((warp == 1 || warp == 2) && lane == 0 && leader) {
+            // ----------------------------------- MMA (even CTA only, two threads)
+            // Thread q issues the K blocks kc with kc % 2 == q (independent partials,
+            // each in its own TMEM buffer; with STAGES and NBUF even each stage and
+            // buffer belongs to one thread, so its parity waits stay in order); one
+            // multicast commit per K block.
+            const int q = warp - 1;
+            const int my_tiles = pair < num_tiles ? (num_tiles - 1 - pair) / num_pairs + 1 : 0;
+            const int total = my_tiles * Kb;
             const uint32_t a0 = smem_u32(smem + L::kOffA);
             const uint32_t b0 = smem_u32(smem + L::kOffB);
-            for (int t = pair; t < num_tiles && ok; t += num_pairs) {
-                for (int kb = 0; kb < Kb; ++kb, ++it, ++kc) {
-                    const int s = it % STAGES;
-                    const uint32_t u = static_cast<uint32_t>(it / STAGES);
-                    const int buf = kc % NBUF;
-                    const uint32_t v = static_cast<uint32_t>(kc / NBUF);
-                    if (!mbar_wait(&tempty[buf], (v & 1u) ^ 1u, abort_flag, p.timeout_ns) ||
-                        !mbar_wait(&full[s], u & 1u, abort_flag, p.timeout_ns)) {
-                        record_failure(p.status, kStatusTimeout, 22, it);
-                        *abort_flag = 1;
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint64_t adesc = sdesc_kmajor_sw128(a0 + s * L::kABytes);
-                    const uint64_t bdesc = sdesc_kmajor_sw128(b0 + s * L::kBBytes);
-                    const uint32_t d = tmem_base + static_cast<uint32_t>(buf * BN);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        umma_e4m3_pair(d, adesc + 2u * k, bdesc + 2u * k, kIdesc, k > 0 ? 1u : 0u);
-                    umma_commit_pair(&empty[s], 0x3);
-                    umma_commit_pair(&tfull[buf], 0x3);
+            int last = -1;
+            for (int kc = q; kc < total; kc += 2) {
+                const int s = kc % STAGES;
+                const uint32_t u = static_cast<uint32_t>(kc / STAGES);
+                const int buf = kc % NBUF;
+                const uint32_t v = static_cast<uint32_t>(kc / NBUF);
+                if (!mbar_wait(&tempty[buf], (v & 1u) ^ 1u, abort_flag, p.timeout_ns) ||
+                    !mbar_wait(&full[s], u & 1u, abort_flag, p.timeout_ns)) {
+                    record_failure(p.status, kStatusTimeout, 22, kc);
+                    *abort_flag = 1;
+                    break;
                 }
+                tc_fence_after();
+                const uint64_t adesc = sdesc_kmajor_sw128(a0 + s * L::kABytes);
+                const uint64_t bdesc = sdesc_kmajor_sw128(b0 + s * L::kBBytes);
+                const uint32_t d = tmem_base + static_cast<uint32_t>(buf * BN);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    umma_e4m3_pair(d, adesc + 2u * k, bdesc + 2u * k, kIdesc, k > 0 ? 1u : 0u);
+                umma_commit_pair(&tfull[buf], 0x3);
+                last = kc;
             }
-            if (kc > 0) {
+            if (last >= 0) {
                 const int never = 0;
-                const int last = kc - 1;
-                if (!mbar_wait(&tfull[last % NBUF], static_cast<uint32_t>(last / NBUF) & 1u, &never, p.timeout_ns))
-                    record_failure(p.status, kStatusTimeout, 22, -1);
+                umma_commit_pair(&mdone[q], 0x1);  // this CTA's barrier only
+                if (!mbar_wait(&mdone[q], 0, &never, p.timeout_ns)) record_failure(p.status, kStatusTimeout, 22, -1);
             }
         }
     } else {
-        regs_alloc<kPairRegsEpilogue>();
+        regs_alloc<pair_regs_epilogue<BN>()>();
         // -------------------------------------------------- epilogue (both CTAs)
         const int ew = warp - 4;
         const int quarter = warp & 3;
@@ -237,21 +244,31 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                     break;
                 }
                 tc_fence_after();
+                // the pair's MMAs of this K block are complete: this CTA's stage is free
+                if (ew == 0 && lane == 0) mbar_arrive(&empty[kc % STAGES]);
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                        static_cast<uint32_t>(buf * BN + half * kColsPerWarp);
+                constexpr int kChunks = kColsPerWarp / 16;
+                uint32_t r0[16], r1[16];
+                tmem_load16_async(taddr, r0);
+                tmem_wait16(r0);
 #pragma unroll
-                for (int c = 0; c < kColsPerWarp / 64; ++c) {
-                    float part[64];
-                    tmem_load64(taddr + c * 64, part);
-                    if (c == kColsPerWarp / 64 - 1) {
+                for (int c = 0; c < kChunks; ++c) {
+                    uint32_t(&cur)[16] = (c & 1) ? r1 : r0;
+                    uint32_t(&nxt)[16] = (c & 1) ? r0 : r1;
+                    if (c + 1 < kChunks) {
+                        tmem_load16_async(taddr + (c + 1) * 16, nxt);
+                    } else {
                         // this CTA's columns of the buffer are in registers: release them
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive_cluster(tempty0 + 8u * buf);
                     }
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        acc[c * 32 + i] = __ffma2_rn(make_float2(part[2 * i], part[2 * i + 1]), s2, acc[c * 32 + i]);
+                    for (int i = 0; i < 8; ++i)
+                        acc[c * 8 + i] = __ffma2_rn(make_float2(__uint_as_float(cur[2 * i]), __uint_as_float(cur[2 * i + 1])),
+                                                    s2, acc[c * 8 + i]);
+                    if (c + 1 < kChunks) tmem_wait16(nxt);
                 }
             }
             if (!ok) break;
@@ -297,6 +314,7 @@ template <int BN, int STAGES, int NBUF>
 static dg_status_t launch_pair_impl(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream) {
     using L = PairSmem<BN, STAGES, NBUF>;
     static_assert(L::kDynamicBytes <= 232448, "shared memory budget");
+    static_assert(STAGES % 2 == 0 && NBUF % 2 == 0, "each MMA thread must own its stages and buffers");
     CUtensorMap tmA, tmB, tmC;
     dg_status_t st;
     st = make_tmap_2d(&tmA, a.A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.M, a.K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -343,7 +361,7 @@ static dg_status_t launch_pair_impl(const GemmArgs &a, const DeviceInfo &dev, cu
             return DG_ERR_CUDA;
         cudaFuncAttributes fa;
         if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return DG_ERR_CUDA;
-        if (128 * kPairRegsProducer + 256 * kPairRegsEpilogue > kPairThreads * fa.numRegs) return DG_ERR_CUDA;
+        if (128 * pair_regs_producer<BN>() + 256 * pair_regs_epilogue<BN>() > kPairThreads * fa.numRegs) return DG_ERR_CUDA;
         cfg.gridDim = dim3(static_cast<unsigned>(dev.num_sms & ~1), 1, 1);
         int clusters = 0;
         if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg) != cudaSuccess || clusters < 1)

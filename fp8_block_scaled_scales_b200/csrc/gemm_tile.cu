@@ -9,25 +9,26 @@
 // registers ("segmented accumulation", 2kiu.com/news/5461879 §3.3), in ascending kb.
 //
 // Roles (one CTA per SM, 12 warps; warpgroup 0 gives registers to the two
-// epilogue warpgroups with setmaxnreg: 128 x 40 + 256 x 232 = 384 x 168, the
-// registers the block is launched with -- the split must not exceed them, or
-// setmaxnreg.inc would wait forever; the launcher checks the compiled count):
+// epilogue warpgroups with setmaxnreg (128 x 56 + 256 x 224 = 384 x 168, the
+// registers the block is launched with, for 256-column tiles) -- a split above
+// them would make setmaxnreg.inc wait forever; the launcher checks the count):
 //   warp 0      TMA producer: 128-K slabs of A (128 rows) and B (BN rows) into a
 //               STAGES-deep ring of 128-byte-swizzled shared-memory stages
 //               (demingchina.com/news/60142 §3.3 producer/consumer split, §4.2
 //               swizzle, §4.3 multi-stage ring).
-//   warp 1      MMA issuer: one thread issues four tcgen05.mma (K = 32 each) per
-//               slab into one of two TMEM partial buffers, then commits to the
-//               stage's "empty" barrier and the buffer's "full" barrier.
-//   warps 2-3   idle.
-//   warps 4-11  epilogue: per kb, tcgen05.ld the partial 64 columns at a time,
+//   warps 1-2   MMA issuers: one thread each, alternating K blocks; per K block
+//               four tcgen05.mma (K = 32 each) into that K block's TMEM partial
+//               buffer, then one commit to the buffer's "full" barrier.
+//   warp 3      idle.
+//   warps 4-11  epilogue: per kb, free the shared-memory stage, tcgen05.ld the
+//               partial 16 columns at a time (software-pipelined against the FMAs),
 //               release the TMEM buffer as soon as the last load has landed, and
 //               acc += s * P_kb with packed FP32 FMAs; after the last kb, round to
 //               BF16, stage in swizzled shared memory and TMA-store.  Warp w reads
 //               TMEM lanes 32*(w%4).. (the lane quarter its warp id allows) and
 //               columns half (w-4)/4 of the tile.
-// While the epilogue works on buffer b the MMA warp fills buffer b^1, so the
-// tensor cores run ahead by one K block; at a tile boundary they run into the
+// While the epilogue works on buffer b the MMA threads fill the next buffer, so
+// the tensor cores run ahead by NBUF - 1 K blocks; at a tile boundary they run into the
 // next tile while the epilogue writes the previous tile's output.
 //
 // Grouped form: m-blocks run over the padded concatenation of the experts' rows;
@@ -59,9 +60,12 @@ struct TileParams {
 
 constexpr int kTileThreads = 384;
 constexpr int kRegsLaunch = 168;    // 65536 / 384 rounded down to a multiple of 8
-constexpr int kRegsProducer = 40;   // warpgroup 0 (TMA, MMA, two idle warps)
-constexpr int kRegsEpilogue = 232;  // warpgroups 1 and 2
-static_assert(128 * kRegsProducer + 256 * kRegsEpilogue <= kTileThreads * kRegsLaunch,
+// setmaxnreg split: warpgroup 0 (TMA producer, two MMA issuers, an idle warp) and the two
+// epilogue warpgroups; the 256-column epilogue needs the larger share.
+template <int BN> __host__ __device__ constexpr int regs_producer() { return BN == 256 ? 56 : 64; }
+template <int BN> __host__ __device__ constexpr int regs_epilogue() { return BN == 256 ? 224 : 216; }
+static_assert(128 * regs_producer<256>() + 256 * regs_epilogue<256>() <= kTileThreads * kRegsLaunch &&
+                  128 * regs_producer<128>() + 256 * regs_epilogue<128>() <= kTileThreads * kRegsLaunch,
               "setmaxnreg split exceeds the registers the block is launched with");
 constexpr int kRasterM = 8;  // m-blocks per raster group (L2 reuse of B tiles)
 
@@ -93,7 +97,7 @@ struct TileSmem {
     static constexpr uint32_t kOffB = kOffA + STAGES * kABytes;
     static constexpr uint32_t kOffC = kOffB + STAGES * kBBytes;
     static constexpr uint32_t kOffBar = kOffC + 8 * kCBoxBytes;
-    static constexpr uint32_t kNumBars = 2 * STAGES + 2 * NBUF;
+    static constexpr uint32_t kNumBars = 2 * STAGES + 2 * NBUF + 2;
     static constexpr uint32_t kOffMisc = kOffBar + 8 * kNumBars;
     static constexpr uint32_t kBytes = kOffMisc + 16;
     static constexpr uint32_t kDynamicBytes = kBytes + 1024;  // slack for 1024-byte alignment
@@ -104,7 +108,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
     tile_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, const TileParams p) {
     using L = TileSmem<BN, STAGES, NBUF>;
-    constexpr int kColsPerWarp = BN / 2;
+        constexpr int kColsPerWarp = BN / 2;
     constexpr uint32_t kTmemCols = tmem_cols_for(NBUF * BN);
     constexpr uint32_t kIdesc = idesc_e4m3_f32(128, BN);
 
@@ -114,6 +118,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
     uint64_t *empty = full + STAGES;
     uint64_t *tfull = empty + STAGES;
     uint64_t *tempty = tfull + NBUF;
+    uint64_t *mdone = tempty + NBUF;  // one per MMA thread: all its MMAs complete
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
 
@@ -125,6 +130,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
+        for (int q = 0; q < 2; ++q) mbar_init(&mdone[q], 1);
         for (int b = 0; b < NBUF; ++b) {
             mbar_init(&tfull[b], 1);
             mbar_init(&tempty[b], 8);
@@ -149,7 +155,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
     const int Kb = p.Kb;
 
     if (warp < 4) {
-        regs_dealloc<kRegsProducer>();
+        regs_dealloc<regs_producer<BN>()>();
         if (warp == 0 && lane == 0) {
             // ------------------------------------------------------------ producer
             uint32_t issued = 0, parity_bits = 0;
@@ -183,46 +189,54 @@ __global__ void __launch_bounds__(kTileThreads, 1)
                 if (issued & (1u << s))
                     if (!mbar_wait(&full[s], (parity_bits >> s) & 1u, &never, p.timeout_ns))
                         record_failure(p.status, kStatusTimeout, 0, -1 - s);
-        } else if (warp == 1 && lane == 0) {
-            // ----------------------------------------------------------------- MMA
-            int it = 0, kc = 0;
-            bool ok = true;
+        } else if ((warp == 1 || warp == 2) && lane == 0) {
+            // ------------------------------------------------------- MMA (two threads)
+            // Thread q issues the K blocks kc with kc % 2 == q.  Every K block's
+            // partial starts from zero in its own TMEM buffer, so the two streams are
+            // independent, and each issuer's barrier waits and commits hide behind the
+            // other's MMAs.  With STAGES and NBUF even, every stage and every buffer
+            // belongs to one thread, which therefore waits on each barrier's phases in
+            // order -- a parity wait is only sound one phase ahead.  One commit per K
+            // block: the epilogue frees the shared-memory stage once it has seen the
+            // buffer full.
+            const int q = warp - 1;
+            const int my_tiles = static_cast<int>(blockIdx.x) < num_tiles
+                                     ? (num_tiles - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
+                                     : 0;
+            const int total = my_tiles * Kb;
             const uint32_t a0 = smem_u32(smem + L::kOffA);
             const uint32_t b0 = smem_u32(smem + L::kOffB);
-            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-                for (int kb = 0; kb < Kb; ++kb, ++it, ++kc) {
-                    const int s = it % STAGES;
-                    const uint32_t u = static_cast<uint32_t>(it / STAGES);
-                    const int buf = kc % NBUF;
-                    const uint32_t v = static_cast<uint32_t>(kc / NBUF);
-                    if (!mbar_wait(&tempty[buf], (v & 1u) ^ 1u, abort_flag, p.timeout_ns) ||
-                        !mbar_wait(&full[s], u & 1u, abort_flag, p.timeout_ns)) {
-                        record_failure(p.status, kStatusTimeout, 1, it);
-                        *abort_flag = 1;
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint64_t adesc = sdesc_kmajor_sw128(a0 + s * L::kABytes);
-                    const uint64_t bdesc = sdesc_kmajor_sw128(b0 + s * L::kBBytes);
-                    const uint32_t d = tmem_base + static_cast<uint32_t>(buf * BN);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)  // 32 bytes of K per instruction = +2 in the address field
-                        umma_e4m3(d, adesc + 2u * k, bdesc + 2u * k, kIdesc, k > 0 ? 1u : 0u);
-                    umma_commit(&empty[s]);
-                    umma_commit(&tfull[buf]);
+            int last = -1;
+            for (int kc = q; kc < total; kc += 2) {
+                const int s = kc % STAGES;
+                const uint32_t u = static_cast<uint32_t>(kc / STAGES);
+                const int buf = kc % NBUF;
+                const uint32_t v = static_cast<uint32_t>(kc / NBUF);
+                if (!mbar_wait(&tempty[buf], (v & 1u) ^ 1u, abort_flag, p.timeout_ns) ||
+                    !mbar_wait(&full[s], u & 1u, abort_flag, p.timeout_ns)) {
+                    record_failure(p.status, kStatusTimeout, 1, kc);
+                    *abort_flag = 1;
+                    break;
                 }
+                tc_fence_after();
+                const uint64_t adesc = sdesc_kmajor_sw128(a0 + s * L::kABytes);
+                const uint64_t bdesc = sdesc_kmajor_sw128(b0 + s * L::kBBytes);
+                const uint32_t d = tmem_base + static_cast<uint32_t>(buf * BN);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)  // 32 bytes of K per instruction = +2 in the address field
+                    umma_e4m3(d, adesc + 2u * k, bdesc + 2u * k, kIdesc, k > 0 ? 1u : 0u);
+                umma_commit(&tfull[buf]);
+                last = kc;
             }
             // the tensor memory may only be released once every MMA issued is done
-            if (kc > 0) {
+            if (last >= 0) {
                 const int never = 0;
-                const int last = kc - 1;
-                if (!mbar_wait(&tfull[last % NBUF], static_cast<uint32_t>(last / NBUF) & 1u, &never, p.timeout_ns))
-                    record_failure(p.status, kStatusTimeout, 1, -1);
+                umma_commit(&mdone[q]);
+                if (!mbar_wait(&mdone[q], 0, &never, p.timeout_ns)) record_failure(p.status, kStatusTimeout, 1, -1);
             }
         }
     } else {
-        regs_alloc<kRegsEpilogue>();
+        regs_alloc<regs_epilogue<BN>()>();
         // -------------------------------------------------------------- epilogue
         const int ew = warp - 4;
         const int quarter = warp & 3;
@@ -256,21 +270,32 @@ __global__ void __launch_bounds__(kTileThreads, 1)
                     break;
                 }
                 tc_fence_after();
+                // the MMAs of this K block are complete, so its shared-memory stage is free
+                if (ew == 0 && lane == 0) mbar_arrive(&empty[kc % STAGES]);
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                        static_cast<uint32_t>(buf * BN + half * kColsPerWarp);
+                // 16 columns at a time: the load of chunk c+1 is in flight while chunk c
+                // is promoted; the buffer is handed back as soon as the last load landed.
+                constexpr int kChunks = kColsPerWarp / 16;
+                uint32_t r0[16], r1[16];
+                tmem_load16_async(taddr, r0);
+                tmem_wait16(r0);
 #pragma unroll
-                for (int c = 0; c < kColsPerWarp / 64; ++c) {
-                    float part[64];
-                    tmem_load64(taddr + c * 64, part);
-                    if (c == kColsPerWarp / 64 - 1) {
-                        // every column of this buffer is in registers: hand it back
+                for (int c = 0; c < kChunks; ++c) {
+                    uint32_t(&cur)[16] = (c & 1) ? r1 : r0;
+                    uint32_t(&nxt)[16] = (c & 1) ? r0 : r1;
+                    if (c + 1 < kChunks) {
+                        tmem_load16_async(taddr + (c + 1) * 16, nxt);
+                    } else {
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&tempty[buf]);
                     }
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        acc[c * 32 + i] = __ffma2_rn(make_float2(part[2 * i], part[2 * i + 1]), s2, acc[c * 32 + i]);
+                    for (int i = 0; i < 8; ++i)
+                        acc[c * 8 + i] = __ffma2_rn(make_float2(__uint_as_float(cur[2 * i]), __uint_as_float(cur[2 * i + 1])),
+                                                    s2, acc[c * 8 + i]);
+                    if (c + 1 < kChunks) tmem_wait16(nxt);
                 }
             }
             if (!ok) break;
@@ -315,6 +340,7 @@ template <int BN, bool GROUPED, int STAGES, int NBUF>
 static dg_status_t launch_tile_impl(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream) {
     using L = TileSmem<BN, STAGES, NBUF>;
     static_assert(L::kDynamicBytes <= 232448, "shared memory budget");
+    static_assert(STAGES % 2 == 0 && NBUF % 2 == 0, "each MMA thread must own its stages and buffers");
     CUtensorMap tmA, tmB, tmC;
     const uint64_t b_rows = GROUPED ? static_cast<uint64_t>(a.G) * a.N : static_cast<uint64_t>(a.N);
     dg_status_t st;
@@ -355,7 +381,7 @@ static dg_status_t launch_tile_impl(const GemmArgs &a, const DeviceInfo &dev, cu
         // the register split inside the kernel must fit what a launch provides
         cudaFuncAttributes fa;
         if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return DG_ERR_CUDA;
-        if (128 * kRegsProducer + 256 * kRegsEpilogue > kTileThreads * fa.numRegs) return DG_ERR_CUDA;
+        if (128 * regs_producer<BN>() + 256 * regs_epilogue<BN>() > kTileThreads * fa.numRegs) return DG_ERR_CUDA;
         configured_device = device;
     }
     const int64_t tiles = static_cast<int64_t>(p.num_m_cap) * p.num_n_tiles;
