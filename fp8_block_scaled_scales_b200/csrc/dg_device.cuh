@@ -429,6 +429,11 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t *bar, uint16_t cta_mas
         : "memory");
 }
 
+// Named barrier over `count` threads (a multiple of 32) of the CTA.
+__device__ __forceinline__ void bar_named_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // Register-budget hints for warp-specialised kernels.
 template <int N>
 __device__ __forceinline__ void regs_dealloc() {

@@ -74,7 +74,7 @@ __device__ __forceinline__ void tmem_load16(uint32_t taddr, float (&v)[16]) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-template <int MP, int STAGES>
+template <int MP, int STAGES, int NBUF>
 struct SkinnySmem {
     static constexpr uint32_t kWBytes = 128 * 128;  // weight slab: 128 rows of B x 128 K
     static constexpr uint32_t kXBytes = MP * 128;   // token slab: MP rows of A x 128 K
@@ -84,17 +84,24 @@ struct SkinnySmem {
     static constexpr uint32_t kRedBytes = MP * 128 * 4;  // FP32 partial, [MP][128]
     static constexpr uint32_t kDataBytes = kStageEnd > kRedBytes ? kStageEnd : kRedBytes;
     static constexpr uint32_t kOffBar = kDataBytes;
-    static constexpr uint32_t kOffMisc = kOffBar + 8 * (2 * STAGES + 4);
+    static constexpr uint32_t kOffMisc = kOffBar + 8 * (2 * STAGES + 2 * NBUF + 2);
     static constexpr uint32_t kBytes = kOffMisc + 16;
     static constexpr uint32_t kDynamicBytes = kBytes + 1024;
 };
 
-template <int MP, int STAGES>
+// All threads of the cluster; the arrival does not order earlier memory accesses
+// (used where every shared-memory read the peers depend on has already returned).
+__device__ __forceinline__ void cluster_sync_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
+}
+
+template <int MP, int STAGES, int NBUF>
 __global__ void __launch_bounds__(kSkinnyThreads, 1)
     skinny_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                        const SkinnyParams p) {
-    using L = SkinnySmem<MP, STAGES>;
-    constexpr uint32_t kTmemCols = (2 * MP < 32) ? 32 : 2 * MP;
+    using L = SkinnySmem<MP, STAGES, NBUF>;
+    static_assert(STAGES % 2 == 0 && NBUF % 2 == 0, "each MMA thread must own its stages and buffers");
+    constexpr uint32_t kTmemCols = tmem_cols_for(NBUF * MP);
     constexpr uint32_t kIdesc = idesc_e4m3_f32(128, MP);
 
     extern __shared__ uint8_t smem_raw[];
@@ -102,7 +109,8 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
     uint64_t *empty = full + STAGES;
     uint64_t *tfull = empty + STAGES;
-    uint64_t *tempty = tfull + 2;
+    uint64_t *tempty = tfull + NBUF;
+    uint64_t *mdone = tempty + NBUF;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
     float *red = reinterpret_cast<float *>(smem);  // reuses the stage memory after the K loop
@@ -121,16 +129,17 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < NBUF; ++b) {
             mbar_init(&tfull[b], 1);
             mbar_init(&tempty[b], 4);
         }
+        for (int q = 0; q < 2; ++q) mbar_init(&mdone[q], 1);
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmW);
         tma_prefetch_desc(&tmX);
     }
-    if (warp == 1) {
+    if (warp == 3) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
@@ -162,16 +171,19 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
             if (issued & (1u << s))
                 if (!mbar_wait(&full[s], (parity_bits >> s) & 1u, &never, p.timeout_ns))
                     record_failure(p.status, kStatusTimeout, 10, -1 - s);
-    } else if (warp == 1 && lane == 0) {
-        // ------------------------------------------------------------------- MMA
+    } else if ((warp == 1 || warp == 2) && lane == 0) {
+        // -------------------------------------------------- MMA (two threads)
+        // Thread q issues K blocks i with i % 2 == q; with STAGES and NBUF even
+        // each stage and buffer belongs to one thread (in-order parity waits).
+        const int q = warp - 1;
         const uint32_t w0 = smem_u32(smem + L::kOffW);
         const uint32_t x0 = smem_u32(smem + L::kOffX);
-        int done = 0;
-        for (int i = 0; i < nkb; ++i) {
+        int last = -1;
+        for (int i = q; i < nkb; i += 2) {
             const int s = i % STAGES;
             const uint32_t u = static_cast<uint32_t>(i / STAGES);
-            const int buf = i & 1;
-            const uint32_t v = static_cast<uint32_t>(i >> 1);
+            const int buf = i % NBUF;
+            const uint32_t v = static_cast<uint32_t>(i / NBUF);
             if (!mbar_wait(&tempty[buf], (v & 1u) ^ 1u, abort_flag, p.timeout_ns) ||
                 !mbar_wait(&full[s], u & 1u, abort_flag, p.timeout_ns)) {
                 record_failure(p.status, kStatusTimeout, 11, i);
@@ -184,68 +196,70 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
             const uint32_t d = tmem_base + static_cast<uint32_t>(buf * MP);
 #pragma unroll
             for (int k = 0; k < 4; ++k) umma_e4m3(d, wdesc + 2u * k, xdesc + 2u * k, kIdesc, k > 0 ? 1u : 0u);
-            umma_commit(&empty[s]);
             umma_commit(&tfull[buf]);
-            done = i + 1;
+            last = i;
         }
-        if (done > 0) {
+        if (last >= 0) {
             const int never = 0;
-            const int last = done - 1;
-            if (!mbar_wait(&tfull[last & 1], static_cast<uint32_t>(last >> 1) & 1u, &never, p.timeout_ns))
-                record_failure(p.status, kStatusTimeout, 11, -1);
+            umma_commit(&mdone[q]);
+            if (!mbar_wait(&mdone[q], 0, &never, p.timeout_ns)) record_failure(p.status, kStatusTimeout, 11, -1);
         }
     } else if (warp >= 4) {
         // -------------------------------------------------------------- epilogue
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;  // output column n = nb*128 + row
-        float acc[MP];
+        float2 acc[MP / 2];
 #pragma unroll
-        for (int j = 0; j < MP; ++j) acc[j] = 0.0f;
+        for (int j = 0; j < MP / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
         ScaleStream scales;
         scales.start(p.sA, p.sB + static_cast<int64_t>(nb) * p.Kb, kb0, kb1);
-        bool ok = true;
         for (int i = 0; i < nkb; ++i) {
-            const int buf = i & 1;
-            const uint32_t v = static_cast<uint32_t>(i >> 1);
+            const int buf = i % NBUF;
+            const uint32_t v = static_cast<uint32_t>(i / NBUF);
             const int kb = kb0 + i;
             const float scale = scales.scale(kb, i);
+            const float2 s2 = make_float2(scale, scale);
             if (!mbar_wait(&tfull[buf], v & 1u, abort_flag, p.timeout_ns)) {
                 record_failure(p.status, kStatusTimeout, 12, i);
                 *abort_flag = 1;
-                ok = false;
                 break;
             }
             tc_fence_after();
+            // the MMAs of this K block are done: its stage may be refilled
+            if (quarter == 0 && lane == 0) mbar_arrive(&empty[i % STAGES]);
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                    static_cast<uint32_t>(buf * MP);
-            if constexpr (MP == 16) {
-                float part[16];
-                tmem_load16(taddr, part);
+            constexpr int kChunks = MP / 16;
+            uint32_t r0[16], r1[16];
+            tmem_load16_async(taddr, r0);
+            tmem_wait16(r0);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) acc[j] = fmaf(scale, part[j], acc[j]);
-            } else {
-#pragma unroll
-                for (int c = 0; c < MP / 32; ++c) {
-                    float part[32];
-                    tmem_load32(taddr + c * 32, part);
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) acc[c * 32 + j] = fmaf(scale, part[j], acc[c * 32 + j]);
+            for (int c = 0; c < kChunks; ++c) {
+                uint32_t(&cur)[16] = (c & 1) ? r1 : r0;
+                uint32_t(&nxt)[16] = (c & 1) ? r0 : r1;
+                if (c + 1 < kChunks) {
+                    tmem_load16_async(taddr + (c + 1) * 16, nxt);
+                } else {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&tempty[buf]);
                 }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[buf]);
-        }
-        // Every MMA of this CTA must be complete before the stage memory is reused
-        // for the partial tile: the MMA warp's last commit arrives on tfull.
-        if (ok && nkb > 0) {
-            const int last = nkb - 1;
-            const int never = 0;
-            mbar_wait(&tfull[last & 1], static_cast<uint32_t>(last >> 1) & 1u, &never, p.timeout_ns);
-        }
-        // partial tile, [MP][128]: consecutive threads write consecutive words
 #pragma unroll
-        for (int j = 0; j < MP; ++j) red[j * 128 + row] = acc[j];
+                for (int j = 0; j < 8; ++j)
+                    acc[c * 8 + j] = __ffma2_rn(make_float2(__uint_as_float(cur[2 * j]), __uint_as_float(cur[2 * j + 1])),
+                                                s2, acc[c * 8 + j]);
+                if (c + 1 < kChunks) tmem_wait16(nxt);
+            }
+        }
+        // every MMA of this CTA has completed once the epilogue saw its last tfull
+        // (or the MMA threads drained after a failure), so the stage memory may now
+        // hold the partial tile, [MP][128]: consecutive threads write consecutive words
+        bar_named_sync(1, 128);  // the four epilogue warps: all TMEM reads done
+#pragma unroll
+        for (int j = 0; j < MP / 2; ++j) {
+            red[(2 * j) * 128 + row] = acc[j].x;
+            red[(2 * j + 1) * 128 + row] = acc[j].y;
+        }
     }
 
     // ---------------------------------------------- split-K reduction over the cluster
@@ -277,21 +291,22 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
             }
         }
     }
-    // no CTA may leave while its peers still read its shared memory
+    // no CTA may leave while its peers still read its shared memory; every read a
+    // peer depends on has returned by the time it arrives
     __syncwarp();
-    cluster_sync_all();
+    cluster_sync_relaxed();
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == 3) {
         tc_fence_after();
         tmem_dealloc(tmem_base, kTmemCols);
     }
 }
 
-template <int MP, int STAGES>
+template <int MP, int STAGES, int NBUF>
 static dg_status_t launch_skinny_impl(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream) {
-    using L = SkinnySmem<MP, STAGES>;
+    using L = SkinnySmem<MP, STAGES, NBUF>;
     static_assert(L::kDynamicBytes <= 232448, "shared memory budget");
     CUtensorMap tmW, tmX;
     dg_status_t st = make_tmap_2d(&tmW, a.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.N, a.K, 128, 128,
@@ -300,7 +315,7 @@ static dg_status_t launch_skinny_impl(const GemmArgs &a, const DeviceInfo &dev, 
     st = make_tmap_2d(&tmX, a.A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.M, a.K, MP, 128, CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != DG_OK) return st;
 
-    auto kernel = skinny_gemm_kernel<MP, STAGES>;
+    auto kernel = skinny_gemm_kernel<MP, STAGES, NBUF>;
     static thread_local int configured_device = -1;
     int device = 0;
     cudaGetDevice(&device);
@@ -346,10 +361,10 @@ static dg_status_t launch_skinny_impl(const GemmArgs &a, const DeviceInfo &dev, 
 }
 
 dg_status_t launch_skinny_gemm(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream) {
-    if (a.M <= 16) return launch_skinny_impl<16, 8>(a, dev, stream);
-    if (a.M <= 32) return launch_skinny_impl<32, 8>(a, dev, stream);
-    if (a.M <= 64) return launch_skinny_impl<64, 8>(a, dev, stream);
-    return launch_skinny_impl<128, 6>(a, dev, stream);
+    if (a.M <= 16) return launch_skinny_impl<16, 8, 8>(a, dev, stream);
+    if (a.M <= 32) return launch_skinny_impl<32, 8, 8>(a, dev, stream);
+    if (a.M <= 64) return launch_skinny_impl<64, 8, 8>(a, dev, stream);
+    return launch_skinny_impl<128, 6, 4>(a, dev, stream);
 }
 
 }  // namespace dg

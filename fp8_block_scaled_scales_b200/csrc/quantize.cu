@@ -29,43 +29,49 @@ namespace dg {
 
 constexpr int kQuantThreads = 256;
 
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-// True when y = x * r might not round to the same E4M3 code as fl32(x / s): y is
-// within 6 FP32 ulps of an E4M3 rounding midpoint (bit 19 set, bits 0-18 clear,
-// i.e. bits[19:0] in [0x7FFFA, 0x80006]) or below 2^-6, where E4M3 is subnormal
-// and its midpoints sit at other bit positions.
-__device__ __forceinline__ bool needs_exact(float y) {
-    const uint32_t b = __float_as_uint(y);
-    const bool near_mid = ((b + 0x80006u) & 0xFFFFFu) <= 12u;
-    return near_mid || (fabsf(y) < 0x1p-6f);
-}
-
-__device__ __forceinline__ uint32_t to_e4m3x4(float2 a, float2 b) {
-    const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(a, __NV_SATFINITE, __NV_E4M3);
-    const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(b, __NV_SATFINITE, __NV_E4M3);
-    return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+// Four floats -> four E4M3 codes (round to nearest even, saturating at +-448), the
+// first in the lowest byte.  cvt...e4m3x2 puts its first source operand in the
+// high byte of the 16-bit result.
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+    uint32_t out;
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+        "mov.b32 %0, {lo, hi};\n\t}"
+        : "=r"(out)
+        : "f"(a), "f"(b), "f"(c), "f"(d));
+    return out;
 }
 
 // Eight BF16 (one 16-byte group) -> eight E4M3 codes.
+//
+// y = x * r (r = 1/s correctly rounded) decides the same E4M3 code as fl32(x / s)
+// unless y lies within a few FP32 ulps of an E4M3 rounding midpoint (mantissa bit
+// 19 set and bits 0-18 clear: bits[19:0] in [0x7FFFA, 0x80006]) or below 2^-6,
+// where E4M3 is subnormal and its midpoints sit at other bit positions.  Both
+// conditions are tracked branch-free as running minima over the eight values
+// (distance to the midpoint pattern, and |y|); only when one fires -- rarely --
+// are the eight quotients recomputed with IEEE division.
 __device__ __forceinline__ uint2 quantize8(uint4 v, float s, float2 r2, bool fast_ok) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
     float2 x[4], y[4];
-    bool slow = !fast_ok;
+    uint32_t dmin = 0xFFFFFFFFu;
+    float ymin = 1.0f;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        x[j] = make_float2(bf16_lo(w[j]), bf16_hi(w[j]));
+        x[j] = make_float2(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xFFFF0000u));
         y[j] = __fmul2_rn(x[j], r2);
-        slow |= needs_exact(y[j].x) | needs_exact(y[j].y);
+        dmin = min(dmin, (__float_as_uint(y[j].x) + 0x80006u) & 0xFFFFFu);
+        dmin = min(dmin, (__float_as_uint(y[j].y) + 0x80006u) & 0xFFFFFu);
+        ymin = fminf(ymin, fminf(fabsf(y[j].x), fabsf(y[j].y)));
     }
-    if (__builtin_expect(slow, 0)) {
+    if (__builtin_expect(dmin <= 12u || ymin < 0x1p-6f || !fast_ok, 0)) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) y[j] = make_float2(__fdiv_rn(x[j].x, s), __fdiv_rn(x[j].y, s));
     }
     uint2 out;
-    out.x = to_e4m3x4(y[0], y[1]);
-    out.y = to_e4m3x4(y[2], y[3]);
+    out.x = e4m3x4(y[0].x, y[0].y, y[1].x, y[1].y);
+    out.y = e4m3x4(y[2].x, y[2].y, y[3].x, y[3].y);
     return out;
 }
 
