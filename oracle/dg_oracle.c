@@ -190,10 +190,13 @@ void dgo_quantize_blockwise(const uint16_t *X, int64_t R, int64_t C, int64_t blk
  * below 2^18, and a sum of 128 of them is below 2^25 in magnitude: at most 43
  * significant bits.  The product of two FP32 scales is exact in FP64 (48 bits).
  *
- * A: [M][K] codes, B: [N][K] codes, sA: [ceil(M/128)][K/128], sB: [ceil(N/128)][K/128].
+ * A: [M][K] codes, B: [N][K] codes, sA: [ceil(M/128)][ceil(K/128)],
+ * sB: [ceil(N/128)][ceil(K/128)].
  * Only rows m in rows[0..nrows) and columns n in cols[0..ncols) are evaluated
  * (pass rows == NULL / cols == NULL for all); out is [nrows][ncols].
- * K must be a multiple of blk.
+ * K need not be a multiple of blk: the last K block then holds the K % blk
+ * columns that exist and nothing else (each K step clipped to what remains,
+ * demingchina.com/news/60142 §6.3), with its own pair of scales.
  */
 static void decode_rows(const uint8_t *X, int64_t K, int64_t row, double *out, const double *tab)
 {
@@ -207,7 +210,7 @@ void dgo_gemm_ref(const uint8_t *A, const float *sA, const uint8_t *B, const flo
 {
     double tab[256];
     dgo_e4m3_table(tab);
-    int64_t Kb = K / blk;
+    int64_t Kb = (K + blk - 1) / blk;
     if (rows == NULL) nrows = M;
     if (cols == NULL) ncols = N;
     /* decode the needed B rows once */
@@ -229,7 +232,8 @@ void dgo_gemm_ref(const uint8_t *A, const float *sA, const uint8_t *B, const flo
                 double ref = 0.0;
                 for (int64_t kb = 0; kb < Kb; ++kb) {
                     double p = 0.0;
-                    for (int64_t k = kb * blk; k < (kb + 1) * blk; ++k) p += Ad[k] * b[k];
+                    int64_t k1 = (kb + 1) * blk < K ? (kb + 1) * blk : K;
+                    for (int64_t k = kb * blk; k < k1; ++k) p += Ad[k] * b[k];
                     double s = (double)sA[(m / blk) * Kb + kb] * (double)sB[(n / blk) * Kb + kb];
                     ref += s * p;
                 }
@@ -244,7 +248,7 @@ void dgo_gemm_ref(const uint8_t *A, const float *sA, const uint8_t *B, const flo
 /*
  * Grouped-contiguous form: the rows of A (and of C) are the concatenation of the
  * experts' token rows, expert g owning rows [off[g], off[g+1]); expert g's weights
- * are B[g] ([N][K] codes) with scales sB[g] ([ceil(N/128)][K/128]).  A row that
+ * are B[g] ([N][K] codes) with scales sB[g] ([ceil(N/128)][ceil(K/128)]).  A row that
  * belongs to no expert (beyond off[G]) is left untouched in out.
  * Row m uses the plain dense formula against B[g], sB[g] for the g that owns it.
  * rows[0..nrows) lists the rows to evaluate; cols == NULL means all N columns.
@@ -254,7 +258,7 @@ void dgo_grouped_gemm_ref(const uint8_t *A, const float *sA, const uint8_t *B, c
                           const int64_t *rows, int64_t nrows, const int64_t *cols, int64_t ncols,
                           double *out)
 {
-    int64_t Nb = (N + blk - 1) / blk, Kb = K / blk;
+    int64_t Nb = (N + blk - 1) / blk, Kb = (K + blk - 1) / blk;
     if (cols == NULL) ncols = N;
     for (int64_t i = 0; i < nrows; ++i) {
         int64_t m = rows[i];

@@ -132,7 +132,8 @@ def _idx(a, n):
 def gemm_ref(A, sA, B, sB, rows=None, cols=None) -> np.ndarray:
     """FP64 block formula for C = A.B^T at the given rows x cols (all if None).
 
-    A [M][K] codes, sA [ceil(M/128)][K/128], B [N][K] codes, sB [ceil(N/128)][K/128].
+    A [M][K] codes, sA [ceil(M/128)][ceil(K/128)], B [N][K] codes, sB [ceil(N/128)][ceil(K/128)].
+    A K that is not a multiple of 128 ends in a partial K block of the columns present.
     """
     lib = _load()
     A = np.ascontiguousarray(A, dtype=np.uint8)
@@ -141,8 +142,8 @@ def gemm_ref(A, sA, B, sB, rows=None, cols=None) -> np.ndarray:
     sB = np.ascontiguousarray(sB, dtype=np.float32)
     M, K = A.shape
     N, K2 = B.shape
-    assert K == K2 and K % BLK == 0
-    assert sA.shape == (-(-M // BLK), K // BLK) and sB.shape == (-(-N // BLK), K // BLK)
+    assert K == K2 and K > 0
+    assert sA.shape == (-(-M // BLK), -(-K // BLK)) and sB.shape == (-(-N // BLK), -(-K // BLK))
     r, nr = _idx(rows, M)
     c, nc = _idx(cols, N)
     out = np.empty((nr, nc), dtype=np.float64)
@@ -155,7 +156,7 @@ def gemm_ref(A, sA, B, sB, rows=None, cols=None) -> np.ndarray:
 def grouped_gemm_ref(A, sA, B, sB, offsets, rows, cols=None) -> np.ndarray:
     """FP64 block formula for the grouped-contiguous layout at the given rows x cols.
 
-    A [M_total][K], sA [M_total/128][K/128], B [G][N][K], sB [G][ceil(N/128)][K/128],
+    A [M_total][K], sA [M_total/128][ceil(K/128)], B [G][N][K], sB [G][ceil(N/128)][ceil(K/128)],
     offsets int32 [G+1].  Rows owned by no expert come back as NaN.
     """
     lib = _load()

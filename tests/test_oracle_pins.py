@@ -57,7 +57,7 @@ def exact_ref(A, sA, B, sB, with_abs=False):
     summation error bound."""
     M, K = A.shape
     N = B.shape[0]
-    Kb = K // 128
+    Kb = -(-K // 128)  # a partial last block holds the K % 128 columns present
     Ai, Bi = codes_to_int(A), codes_to_int(B)
     out = [[Fraction(0)] * N for _ in range(M)]
     absum = np.zeros((M, N))
@@ -205,18 +205,20 @@ def test_bf16_rounding_matches_torch_on_floats():
 
 # ----------------------------------------------------------------------- GEMM
 @pytest.mark.parametrize("M,N,K,seed", [(1, 1, 128, 0), (7, 5, 256, 1), (130, 129, 384, 2),
-                                        (200, 256, 256, 3), (33, 300, 128, 4)])
+                                        (200, 256, 256, 3), (33, 300, 128, 4),
+                                        # K tails: one partial block, and full blocks + a partial one
+                                        (5, 9, 16, 6), (40, 130, 200, 7), (129, 7, 272, 8)])
 def test_gemm_ref_against_exact_brute_force(M, N, K, seed):
     rng = np.random.default_rng(seed)
+    Kb = -(-K // 128)
     A = random_finite_codes(rng, (M, K))
     B = random_finite_codes(rng, (N, K))
-    sA = random_scales(rng, (-(-M // 128), K // 128))
-    sB = random_scales(rng, (-(-N // 128), K // 128))
+    sA = random_scales(rng, (-(-M // 128), Kb))
+    sB = random_scales(rng, (-(-N // 128), Kb))
     ref = oracle.gemm_ref(A, sA, B, sB)
     exact, absum = exact_ref(A, sA, B, sB, with_abs=True)
     ex = np.array([[float(v) for v in row] for row in exact])
     # FP64 error of a Kb-term sum of exactly-partialled terms: a few ulps of sum|term|
-    Kb = K // 128
     assert np.all(np.abs(ref - ex) <= 2 * (Kb + 1) * 2.0 ** -53 * absum)
     # BF16 output: the oracle's rounding of its FP64 value against the exact rounding
     got = bits_to_f64(oracle.bf16_from_double(ref))
@@ -407,3 +409,30 @@ def test_quantizer_matches_torch_division_and_cast():
     assert np.array_equal(q, want)
     # the all-zero block: scale 1, codes zero with the sign kept
     assert s[0, 0] == 1.0 and q[0, 0] == 0x80 and np.all(q[:128, :128].ravel()[1:] == 0)
+
+
+@pytest.mark.parametrize("K", [16, 112, 144, 400])
+def test_gemm_ref_k_tail_equals_zero_padded_full_blocks(K):
+    """A partial last K block is the full block with zero codes in the missing columns.
+
+    Zero codes add exact zeros to the block partial, so padding A and B with zero
+    columns up to a multiple of 128 (same scales) must give the same FP64 values bit
+    for bit; and the tail block's scale pair must act on the tail columns only."""
+    rng = np.random.default_rng(K)
+    M, N = 70, 150
+    Kb = -(-K // 128)
+    A = random_finite_codes(rng, (M, K))
+    B = random_finite_codes(rng, (N, K))
+    sA = random_scales(rng, (-(-M // 128), Kb))
+    sB = random_scales(rng, (-(-N // 128), Kb))
+    ref = oracle.gemm_ref(A, sA, B, sB)
+    Kp = 128 * Kb
+    Ap = np.zeros((M, Kp), np.uint8); Ap[:, :K] = A
+    Bp = np.zeros((N, Kp), np.uint8); Bp[:, :K] = B
+    assert np.array_equal(oracle.gemm_ref(Ap, sA, Bp, sB), ref)
+    # doubling the tail block's A scales doubles exactly the tail's contribution
+    sA2 = sA.copy(); sA2[:, Kb - 1] *= 2
+    head = np.zeros_like(A); head[:, :128 * (Kb - 1)] = A[:, :128 * (Kb - 1)]
+    tail = oracle.gemm_ref(A, sA2, B, sB) - oracle.gemm_ref(head, sA2, B, sB)
+    tail1 = ref - oracle.gemm_ref(head, sA, B, sB)
+    assert np.allclose(tail, 2 * tail1, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
