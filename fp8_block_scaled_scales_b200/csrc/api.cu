@@ -158,7 +158,7 @@ static dg_status_t check_gemm_common(const uint8_t *A, const float *sA, const ui
 dg_status_t dg_fp8_gemm_blockscaled_select(const uint8_t *A, const float *sA, const uint8_t *B, const float *sB,
                                            void *C_bf16, int64_t M, int64_t N, int64_t K, dg_kernel_t kernel,
                                            cudaStream_t stream) {
-    if (M < 0 || N < 0 || K <= 0 || K % 128 != 0 || N % 16 != 0) return DG_ERR_SHAPE;
+    if (M < 0 || N < 0 || K <= 0 || K % 16 != 0 || N % 16 != 0) return DG_ERR_SHAPE;
     // TMA coordinates are 32-bit signed
     if (M > 0x7FFFFFFFLL || N > 0x7FFFFFFFLL || K > 0x7FFFFFFFLL) return DG_ERR_SHAPE;
     if (kernel != DG_KERNEL_AUTO && kernel != DG_KERNEL_TILE && kernel != DG_KERNEL_SKINNY &&
@@ -187,7 +187,7 @@ dg_status_t dg_fp8_grouped_gemm_contiguous(const uint8_t *A, const float *sA, co
                                            void *C_bf16, const int32_t *group_offsets, int64_t M_total_capacity,
                                            int G, int64_t N, int64_t K, cudaStream_t stream) {
     if (M_total_capacity < 0 || M_total_capacity % 128 != 0 || N < 0 || N % 128 != 0 || K <= 0 ||
-        K % 128 != 0 || G < 1 || G > 1024)
+        K % 16 != 0 || G < 1 || G > 1024)
         return DG_ERR_SHAPE;
     if (M_total_capacity > 0x7FFFFFFFLL || static_cast<int64_t>(G) * N > 0x7FFFFFFFLL || K > 0x7FFFFFFFLL)
         return DG_ERR_SHAPE;

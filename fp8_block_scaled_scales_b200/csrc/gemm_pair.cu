@@ -41,7 +41,7 @@ struct PairParams {
     int num_n_tiles;  // ceil(N / BN)
     int M, N;
     int Nb;           // ceil(N / 128)
-    int Kb;           // K / 128
+    int Kb;           // ceil(K / 128); the last K block may be partial
     uint64_t timeout_ns;
     int *status;
     int debug_flags;
@@ -334,7 +334,7 @@ static dg_status_t launch_pair_impl(const GemmArgs &a, const DeviceInfo &dev, cu
     p.M = static_cast<int>(a.M);
     p.N = static_cast<int>(a.N);
     p.Nb = static_cast<int>((a.N + 127) / 128);
-    p.Kb = static_cast<int>(a.K / 128);
+    p.Kb = static_cast<int>((a.K + 127) / 128);
     p.timeout_ns = ctl.timeout_ns;
     p.status = ctl.status;
     p.debug_flags = ctl.debug_flags;

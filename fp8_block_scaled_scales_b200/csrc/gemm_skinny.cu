@@ -327,7 +327,7 @@ static dg_status_t launch_skinny_impl(const GemmArgs &a, const DeviceInfo &dev, 
         configured_device = device;
     }
 
-    const int Kb = static_cast<int>(a.K / 128);
+    const int Kb = static_cast<int>((a.K + 127) / 128);
     const int Nt = static_cast<int>((a.N + 127) / 128);
     // Split K so that the clusters cover the SMs about once: S in {1,2,4,8}, S <= Kb.
     int S = 1;

@@ -52,7 +52,7 @@ struct TileParams {
     int M;            // rows of A and C (dense: M, grouped: capacity)
     int N;
     int Nb;           // ceil(N / 128)
-    int Kb;           // K / 128
+    int Kb;           // ceil(K / 128); the last K block may be partial
     uint64_t timeout_ns;
     int *status;  // device status word
     int debug_flags;
@@ -365,7 +365,7 @@ static dg_status_t launch_tile_impl(const GemmArgs &a, const DeviceInfo &dev, cu
     p.M = static_cast<int>(a.M);
     p.N = static_cast<int>(a.N);
     p.Nb = static_cast<int>((a.N + 127) / 128);
-    p.Kb = static_cast<int>(a.K / 128);
+    p.Kb = static_cast<int>((a.K + 127) / 128);
     p.timeout_ns = ctl.timeout_ns;
     p.status = ctl.status;
     p.debug_flags = ctl.debug_flags;

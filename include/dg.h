@@ -82,10 +82,14 @@ dg_status_t dg_quantize_blockwise(const void *X_bf16, int64_t rows, int64_t cols
  *   C[m][n] = bf16( sum_kb sA[m/128][kb] * sB[n/128][kb] *
  *                   sum_{k in block kb} A[m][k] * B[n][k] )
  *
- * A  : [M][K] E4M3, 16-byte aligned.     sA : [ceil(M/128)][K/128] FP32.
- * B  : [N][K] E4M3, 16-byte aligned.     sB : [ceil(N/128)][K/128] FP32.
+ * A  : [M][K] E4M3, 16-byte aligned.     sA : [ceil(M/128)][ceil(K/128)] FP32.
+ * B  : [N][K] E4M3, 16-byte aligned.     sB : [ceil(N/128)][ceil(K/128)] FP32.
  * C  : [M][N] BF16 out, 16-byte aligned.
- * M >= 0, N >= 0 with N % 16 == 0, K > 0 with K % 128 == 0.
+ * M >= 0, N >= 0 with N % 16 == 0, K > 0 with K % 16 == 0 (a row is a whole
+ * number of 16-byte units).  When K % 128 != 0 the last K block is partial: it
+ * holds the K % 128 columns present and has its own scales, as
+ * dg_quantize_blockwise produces them (each K step clipped to what remains,
+ * demingchina.com/news/60142 §6.3).
  * M == 0 or N == 0 is a no-op.  M <= 128 takes the skinny split-K kernel,
  * larger M the persistent CTA-pair tile kernel; both compute the same formula.
  */
@@ -102,13 +106,14 @@ dg_status_t dg_fp8_gemm_blockscaled(const uint8_t *A, const float *sA,
  * Padding rows inside an expert's range are computed like real rows (zero rows
  * of A give zero rows of C).  Rows at or beyond off[G] are not written.
  *
- * A  : [M_total_capacity][K] E4M3.        sA : [M_total_capacity/128][K/128] FP32.
- * B  : [G][N][K] E4M3.                    sB : [G][N/128][K/128] FP32.
+ * A  : [M_total_capacity][K] E4M3.        sA : [M_total_capacity/128][ceil(K/128)] FP32.
+ * B  : [G][N][K] E4M3.                    sB : [G][N/128][ceil(K/128)] FP32.
  * C  : [M_total_capacity][N] BF16 out.
  * group_offsets : DEVICE int32 [G+1], off[0] == 0, non-decreasing, each a
  *                 multiple of 128, off[G] <= M_total_capacity.  Read on the
  *                 device, so it may be produced by an earlier kernel on `stream`.
- * M_total_capacity % 128 == 0, 1 <= G <= 1024, N % 128 == 0, K % 128 == 0, K > 0.
+ * M_total_capacity % 128 == 0, 1 <= G <= 1024, N % 128 == 0, K % 16 == 0, K > 0
+ * (a partial last K block as in dg_fp8_gemm_blockscaled).
  * M_total_capacity == 0 or N == 0 is a no-op.
  */
 dg_status_t dg_fp8_grouped_gemm_contiguous(const uint8_t *A, const float *sA,

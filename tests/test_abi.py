@@ -49,7 +49,9 @@ def test_host_validation_without_device(lib):
     assert lib.dg_quantize_blockwise(null, 4, 17, null, null, null) == 2
     assert lib.dg_quantize_blockwise(null, -1, 16, null, null, null) == 2
     assert lib.dg_quantize_blockwise(null, 0, 16, null, null, null) == 0
-    assert lib.dg_fp8_gemm_blockscaled(null, null, null, null, null, 8, 16, 100, null) == 2  # K % 128
+    assert lib.dg_fp8_gemm_blockscaled(null, null, null, null, null, 8, 16, 100, null) == 2  # K % 16
+    assert lib.dg_fp8_gemm_blockscaled(null, null, null, null, null, 8, 16, 112, null) == 1  # K tail ok
+    assert lib.dg_fp8_grouped_gemm_contiguous(null, null, null, null, null, null, 128, 2, 128, 40, null) == 2
     assert lib.dg_fp8_gemm_blockscaled(null, null, null, null, null, 8, 24, 128, null) == 2  # N % 16
     assert lib.dg_fp8_gemm_blockscaled(null, null, null, null, null, 8, 16, 0, null) == 2    # K == 0
     assert lib.dg_fp8_gemm_blockscaled(null, null, null, null, null, 0, 16, 128, null) == 0  # M == 0

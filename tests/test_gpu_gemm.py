@@ -56,6 +56,24 @@ def test_dense_small_m_all_kernels(M, N, K, kernel):
     check(c, ref, None, f"{kernel} {M}x{N}x{K}")
 
 
+KTAIL = [(300, 272, 144), (129, 400, 16), (1000, 1008, 656), (64, 256, 48), (260, 128, 1040),
+         (5, 4096, 4000), (128, 512, 4112)]
+
+
+@pytest.mark.parametrize("M,N,K", KTAIL)
+@pytest.mark.parametrize("kernel", ["tile", "pair", "skinny"])
+def test_dense_k_tail_all_kernels(M, N, K, kernel):
+    """K % 128 != 0: the last K block holds the columns present (TMA zero-fills the rest
+    of the box) and is promoted with its own scales."""
+    if kernel == "skinny" and M > 128:
+        pytest.skip("skinny kernel takes M <= 128")
+    d = inputs.dense_custom(M, N, K, seed=8500 + M + N + K)
+    qa, sa, qb, sb = quantized(d)
+    assert sa.shape[1] == -(-K // 128)
+    c = c_f64(run(qa, sa, qb, sb, kernel=kernel))
+    check(c, oracle.gemm_ref(qa, sa, qb, sb), None, f"{kernel} {M}x{N}x{K}")
+
+
 def test_dense_512_workload():
     d = inputs.dense_512()
     qa, sa, qb, sb = quantized(d)
@@ -70,14 +88,17 @@ def _exact_inputs(M, N, K, seed):
     enc = np.vectorize(lambda x: code_of[abs(float(x))] | (0x80 if x < 0 else 0), otypes=[np.uint8])
     va = rng.choice([-1, 0, 0, 0, 0, 0, 1], size=(M, K))
     vb = rng.choice([-2, -1, 0, 0, 0, 0, 0, 1, 2], size=(N, K))
-    sa = (2.0 ** rng.integers(-1, 2, size=(-(-M // 128), K // 128))).astype(np.float32)
-    sb = (2.0 ** rng.integers(-1, 1, size=(-(-N // 128), K // 128))).astype(np.float32)
+    sa = (2.0 ** rng.integers(-1, 2, size=(-(-M // 128), -(-K // 128)))).astype(np.float32)
+    sb = (2.0 ** rng.integers(-1, 1, size=(-(-N // 128), -(-K // 128)))).astype(np.float32)
     return enc(va), sa, enc(vb), sb
 
 
 @pytest.mark.parametrize("M,N,K,kernel", [(300, 400, 256, "tile"), (64, 272, 384, "skinny"),
                                           (128, 256, 256, "tile"), (7, 4096, 256, "skinny"),
-                                          (300, 400, 256, "pair"), (520, 128, 384, "pair")])
+                                          (300, 400, 256, "pair"), (520, 128, 384, "pair"),
+                                          # K tails: the last K block is partial
+                                          (300, 400, 208, "pair"), (130, 256, 80, "tile"),
+                                          (7, 4096, 176, "skinny")])
 def test_dense_exact_small_integers_bit_exact(M, N, K, kernel):
     """Integer E4M3 values and power-of-two scales: every step is exact, so the BF16
     output must equal the oracle's exactly."""

@@ -22,7 +22,7 @@ def run(qa, sa, qb, sb, off, capacity=None, fill=None):
     cap = capacity or Mt
     A = torch.zeros((cap, K), dtype=torch.uint8, device="cuda")
     A[:Mt] = dev(qa)
-    SA = torch.ones((cap // 128, K // 128), dtype=torch.float32, device="cuda")
+    SA = torch.ones((cap // 128, -(-K // 128)), dtype=torch.float32, device="cuda")
     SA[:Mt // 128] = dev(sa)
     C = torch.full((cap, qb.shape[1]), fill if fill is not None else 0.0, dtype=torch.bfloat16, device="cuda")
     binding.grouped_gemm_contiguous(A, SA, dev(qb), dev(sb), dev(off), C=C)
@@ -36,6 +36,7 @@ def run(qa, sa, qb, sb, off, capacity=None, fill=None):
     (3, 384, 640, [1, 300, 0]),
     (1, 128, 128, [77]),
     (6, 512, 384, [0, 0, 129, 64, 0, 256]),
+    (2, 256, 208, [130, 60]),  # K tail: partial last K block
 ])
 def test_grouped_small_full_compare(G, N, K, counts):
     w = inputs.grouped_custom(G, N, K, counts, seed=9000 + G + N)
