@@ -38,6 +38,7 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
+FUSED_MAX_M = 32  # the library quantizes A inside the skinny GEMM up to this M
 L2_FLUSH_BYTES = 256 << 20
 FP8_OVER_BF16 = 2.0  # nominal dense FP8 / BF16 tensor throughput ratio on B200
 
@@ -261,6 +262,7 @@ def run_dg(args):
     flops, gemm_bytes, rows_a, cfg = workload_facts(w)
     grouped = isinstance(w, Grouped)
     skinny = (not grouped) and w.M <= 128
+    fused = skinny and w.M <= FUSED_MAX_M  # one launch: the GEMM quantizes A itself
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream()
 
@@ -273,7 +275,7 @@ def run_dg(args):
         sb = sb.view(w.G, w.N // 128, w.K // 128)
         off = torch.from_numpy(w.offsets).to(dev)
     qa = torch.empty((rows_a, w.K), dtype=torch.uint8, device=dev)
-    sa = torch.empty((-(-rows_a // 128), w.K // 128), dtype=torch.float32, device=dev)
+    sa = torch.empty((-(-rows_a // 128), -(-w.K // 128)), dtype=torch.float32, device=dev)
     C = torch.empty((rows_a, w.N), dtype=torch.bfloat16, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
 
@@ -284,8 +286,11 @@ def run_dg(args):
             binding.gemm_blockscaled(qa, sa, qb, sb, C=C)
 
     def step(x):
-        binding.quantize_blockwise(x, q=qa, s=sa)
-        gemm()
+        if fused:
+            binding.gemm_blockscaled_bf16a(x, qb, sb, C=C, QA=qa, sA=sa)
+        else:
+            binding.quantize_blockwise(x, q=qa, s=sa)
+            gemm()
 
     for _ in range(args.warmup):
         flush.fill_(1)
@@ -312,14 +317,20 @@ def run_dg(args):
         for i in range(K):
             flush.fill_(i)
             ev[i][0].record(stream)
-            binding.quantize_blockwise(A, q=qa, s=sa)
-            ev[i][1].record(stream)
-            gemm()
+            if fused:
+                step(A)  # the fused kernel is the whole step
+            else:
+                binding.quantize_blockwise(A, q=qa, s=sa)
+                ev[i][1].record(stream)
+                gemm()
             ev[i][2].record(stream)
         barrier(world)
     step_ms = [ev[i][0].elapsed_time(ev[i][2]) for i in range(K)]
-    gemm_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
-    quant_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
+    if fused:
+        gemm_ms, quant_ms = step_ms, [0.0] * K
+    else:
+        gemm_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+        quant_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
     if binding.last_device_status() != 0:
         raise SystemExit("device status not OK after the timed region")
     ms_step = max_over_ranks(statistics.mean(step_ms), world)
@@ -348,6 +359,12 @@ def run_dg(args):
     peaks = load_peaks()
     if skinny:
         metric, unit = "FP8 block-scaled GEMM HBM GB/s (skinny M) and % of B200 HBM roofline", "GB/s"
+        if fused:
+            # the fused kernel's algorithmic bytes: BF16 A in, B codes and scales in,
+            # C out, and A's codes and scales out
+            kb = -(-w.K // 128)
+            gemm_bytes = (2 * w.M * w.K + w.N * w.K + 4 * kb * -(-w.N // 128) + 2 * w.M * w.N
+                          + w.M * w.K + 4 * kb)
         per_step = gemm_bytes
         value = world * per_step / (ms_step * 1e-3) / 1e9
         e2e_value = world * per_step / (ms_e2e * 1e-3) / 1e9
@@ -376,12 +393,14 @@ def run_dg(args):
            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 (fp32 accumulate, bf16 out)",
            "data": "synthetic (seeded N(0,1)/N(0,0.02) BF16, quantized per 128x128 block)",
            "config": dict(cfg, l2="flushed before every step (256 MB write outside the events)",
-                          step="quantize A (BF16->E4M3+scales) + block-scaled GEMM; B quantized once",
+                          step=("block-scaled GEMM from BF16 A, quantized inside the GEMM kernel (one launch); "
+                                "B quantized once" if fused else
+                                "quantize A (BF16->E4M3+scales) + block-scaled GEMM; B quantized once"),
                           parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
            "roofline": roof,
            "e2e": {"value": round(e2e_value, 2), "unit": unit,
                    "h2d_bytes_per_step": int(A_host.numel() * 2), "d2h_bytes_per_step": int(C.numel() * 2)},
-           "gpu_launches": 2 * K, "host_enqueue_us_per_step": round(enqueue_s * 1e6, 1)}
+           "gpu_launches": (1 if fused else 2) * K, "host_enqueue_us_per_step": round(enqueue_s * 1e6, 1)}
     cs = clocks.summary()
     if cs is not None:
         out["clocks"] = cs

@@ -22,7 +22,8 @@ STATUS_NAMES = {0: "DG_OK", 1: "DG_ERR_INVALID_ARG", 2: "DG_ERR_SHAPE", 3: "DG_E
 KERNELS = {"auto": 0, "tile": 1, "skinny": 2, "pair": 3}
 
 # every symbol include/dg.h declares
-EXPORTS = ("dg_quantize_blockwise", "dg_fp8_gemm_blockscaled", "dg_fp8_grouped_gemm_contiguous",
+EXPORTS = ("dg_quantize_blockwise", "dg_fp8_gemm_blockscaled", "dg_fp8_gemm_blockscaled_bf16a",
+           "dg_fp8_grouped_gemm_contiguous",
            "dg_fp8_gemm_blockscaled_select", "dg_status_string", "dg_get_last_device_status",
            "dg_version", "dg_test_set_kernel_control")
 
@@ -49,8 +50,10 @@ def lib() -> ctypes.CDLL:
     L.dg_quantize_blockwise.argtypes = [vp, i64, i64, vp, vp, vp]
     L.dg_fp8_gemm_blockscaled.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp]
     L.dg_fp8_gemm_blockscaled_select.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, vp]
+    L.dg_fp8_gemm_blockscaled_bf16a.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp]
     L.dg_fp8_grouped_gemm_contiguous.argtypes = [vp, vp, vp, vp, vp, vp, i64, i32, i64, i64, vp]
     for f in ("dg_quantize_blockwise", "dg_fp8_gemm_blockscaled", "dg_fp8_gemm_blockscaled_select",
+              "dg_fp8_gemm_blockscaled_bf16a",
               "dg_fp8_grouped_gemm_contiguous", "dg_get_last_device_status"):
         getattr(L, f).restype = ctypes.c_int
     L.dg_get_last_device_status.argtypes = [vp]
@@ -115,6 +118,26 @@ def gemm_blockscaled(A, sA, B, sB, C=None, kernel: str = "auto", stream=None):
                                                 KERNELS[kernel], _stream(stream)),
            "dg_fp8_gemm_blockscaled")
     return C
+
+
+def gemm_blockscaled_bf16a(A, B, sB, C=None, QA=None, sA=None, stream=None):
+    """C[M][N] (bf16) = quantize(A)[M][K] . B[N][K]^T from BF16 activations A.
+
+    Returns (C, QA, sA): A's E4M3 codes and 128x128 block scales are outputs too."""
+    M, K = A.shape
+    B = _u8(B)
+    N = B.shape[0]
+    dev = A.device
+    if C is None:
+        C = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    if QA is None:
+        QA = torch.empty((M, K), dtype=torch.uint8, device=dev)
+    if sA is None:
+        sA = torch.empty(((M + 127) // 128, (K + 127) // 128), dtype=torch.float32, device=dev)
+    _check(lib().dg_fp8_gemm_blockscaled_bf16a(_p(A), _p(B), _p(sB), _p(C), _p(_u8(QA)), _p(sA), M, N, K,
+                                               _stream(stream)),
+           "dg_fp8_gemm_blockscaled_bf16a")
+    return C, QA, sA
 
 
 def grouped_gemm_contiguous(A, sA, B, sB, offsets, C=None, stream=None):

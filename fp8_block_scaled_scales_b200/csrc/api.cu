@@ -183,6 +183,29 @@ dg_status_t dg_fp8_gemm_blockscaled(const uint8_t *A, const float *sA, const uin
     return dg_fp8_gemm_blockscaled_select(A, sA, B, sB, C_bf16, M, N, K, DG_KERNEL_AUTO, stream);
 }
 
+dg_status_t dg_fp8_gemm_blockscaled_bf16a(const void *A_bf16, const uint8_t *B, const float *sB, void *C_bf16,
+                                          uint8_t *QA, float *sA, int64_t M, int64_t N, int64_t K,
+                                          cudaStream_t stream) {
+    if (M < 0 || N < 0 || K <= 0 || K % 16 != 0 || N % 16 != 0) return DG_ERR_SHAPE;
+    if (M > 0x7FFFFFFFLL || N > 0x7FFFFFFFLL || K > 0x7FFFFFFFLL) return DG_ERR_SHAPE;
+    if (M == 0 || N == 0) return DG_OK;
+    if (!A_bf16) return DG_ERR_INVALID_ARG;
+    dg_status_t st = check_gemm_common(QA, sA, B, sB, C_bf16);
+    if (st != DG_OK) return st;
+    if (!aligned(A_bf16, 16)) return DG_ERR_ALIGNMENT;
+    DeviceInfo dev;
+    st = current_device(&dev, nullptr);
+    if (st != DG_OK) return st;
+    if (M <= kFusedMaxM) {
+        // one launch: the skinny kernel quantizes A itself and writes QA, sA on the way
+        GemmArgs a = {QA, sA, B, sB, C_bf16, nullptr, M, N, K, 0};
+        return launch_skinny_gemm_fused(a, A_bf16, QA, sA, dev, stream);
+    }
+    st = launch_quantize(A_bf16, M, K, QA, sA, dev, stream);
+    if (st != DG_OK) return st;
+    return dg_fp8_gemm_blockscaled_select(QA, sA, B, sB, C_bf16, M, N, K, DG_KERNEL_AUTO, stream);
+}
+
 dg_status_t dg_fp8_grouped_gemm_contiguous(const uint8_t *A, const float *sA, const uint8_t *B, const float *sB,
                                            void *C_bf16, const int32_t *group_offsets, int64_t M_total_capacity,
                                            int G, int64_t N, int64_t K, cudaStream_t stream) {

@@ -332,10 +332,11 @@ struct ScaleStream {
 
     __device__ __forceinline__ float load(int base) const {
         const int k = base + static_cast<int>(threadIdx.x & 31u);
-        return k < kb_end ? __ldg(a + k) * __ldg(b + k) : 0.0f;
+        return k < kb_end ? (a ? __ldg(a + k) : 1.0f) * __ldg(b + k) : 0.0f;
     }
 
-    // a_row, b_row point at K block 0 of the tile's sA and sB rows; K blocks [kb_begin, end)
+    // a_row, b_row point at K block 0 of the tile's sA and sB rows; K blocks [kb_begin, end).
+    // A null a_row stands for scales of 1 (the caller multiplies the A scale in itself).
     __device__ __forceinline__ void start(const float *a_row, const float *b_row, int kb_begin, int end) {
         a = a_row;
         b = b_row;

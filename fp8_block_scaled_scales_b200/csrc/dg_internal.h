@@ -52,6 +52,12 @@ dg_status_t launch_tile_gemm(const GemmArgs &a, bool grouped, const DeviceInfo &
 dg_status_t launch_pair_gemm(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream);
 dg_status_t launch_pair_gemm_n128(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream);
 dg_status_t launch_skinny_gemm(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream);
+// M <= kFusedMaxM with BF16 A quantized inside the GEMM; a.A and a.sA are unused.
+// Above it every N block's CTAs would repeat too much of the quantization, and the
+// block quantizer followed by the FP8 GEMM is faster.
+constexpr int64_t kFusedMaxM = 32;
+dg_status_t launch_skinny_gemm_fused(const GemmArgs &a, const void *A_bf16, uint8_t *qa_out, float *sa_out,
+                                     const DeviceInfo &dev, cudaStream_t stream);
 dg_status_t launch_quantize(const void *X, int64_t rows, int64_t cols, uint8_t *Q, float *S,
                             const DeviceInfo &dev, cudaStream_t stream);
 

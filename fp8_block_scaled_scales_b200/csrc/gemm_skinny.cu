@@ -15,24 +15,41 @@
 // partials of its 128/S columns in rank order 0..S-1 through distributed shared
 // memory and writes them as BF16.  The order is fixed, so the result is
 // deterministic (no float atomics; demingchina.com/news/60142 §6.4).
+//
+// Fused activation quantization (FUSED): A arrives as BF16 (TMA brings each K
+// block's M x 128 slab into a ring) and four more warps quantize it per 128x128
+// block (for M <= 128 the block of K block kb is rows 0..M-1 x its 128 columns)
+// straight into the MMA's shared-memory stage, in the
+// 128-byte-swizzled K-major layout TMA would have written, with exactly the
+// arithmetic of the block quantizer (quant_e4m3.cuh).  The step before the GEMM
+// thus needs no launch of its own (2kiu.com/news/5461879 §5: activation scales
+// are recomputed on every call).  The CTAs of the first N block also write the
+// codes and scales out, so the caller gets the same Q, S as from the quantizer.
 #include <cuda_bf16.h>
 
 #include "dg_device.cuh"
 #include "dg_internal.h"
+#include "quant_e4m3.cuh"
 
 namespace dg {
 
 struct SkinnyParams {
-    const float *sA;
+    const float *sA;  // null when FUSED (the kernel derives the scales)
     const float *sB;
     __nv_bfloat16 *C;
     int M, N, Kb;
     int splits;
     uint64_t timeout_ns;
     int *status;  // device status word
+    // FUSED only: BF16 A [M][K], and the codes / scales written by the first N block
+    const uint16_t *Xa;
+    int K;
+    uint8_t *qa_out;
+    float *sa_out;
 };
 
-constexpr int kSkinnyThreads = 256;
+template <bool FUSED>
+constexpr int skinny_threads() { return FUSED ? 384 : 256; }
 
 __device__ __forceinline__ uint32_t cluster_rank() {
     uint32_t r;
@@ -74,18 +91,23 @@ __device__ __forceinline__ void tmem_load16(uint32_t taddr, float (&v)[16]) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-template <int MP, int STAGES, int NBUF>
+template <int MP, int STAGES, int NBUF, int RA>
 struct SkinnySmem {
     static constexpr uint32_t kWBytes = 128 * 128;  // weight slab: 128 rows of B x 128 K
     static constexpr uint32_t kXBytes = MP * 128;   // token slab: MP rows of A x 128 K
+    static constexpr uint32_t kABytes = MP * 256;   // FUSED: BF16 token slab, MP rows x 128 K, unswizzled
     static constexpr uint32_t kOffW = 0;
     static constexpr uint32_t kOffX = kOffW + STAGES * kWBytes;
-    static constexpr uint32_t kStageEnd = kOffX + STAGES * kXBytes;
+    static constexpr uint32_t kOffA = kOffX + STAGES * kXBytes;  // FUSED: ring of RA BF16 slabs
+    static constexpr uint32_t kStageEnd = kOffA + RA * kABytes;
     static constexpr uint32_t kRedBytes = MP * 128 * 4;  // FP32 partial, [MP][128]
     static constexpr uint32_t kDataBytes = kStageEnd > kRedBytes ? kStageEnd : kRedBytes;
     static constexpr uint32_t kOffBar = kDataBytes;
-    static constexpr uint32_t kOffMisc = kOffBar + 8 * (2 * STAGES + 2 * NBUF + 2);
-    static constexpr uint32_t kBytes = kOffMisc + 16;
+    static constexpr uint32_t kOffMisc = kOffBar + 8 * (2 * STAGES + 2 * NBUF + 2 + 2 * RA);
+    // misc: TMEM address (0), abort flag (4), FUSED quantizer's stage flag (8)
+    static constexpr uint32_t kOffScaleA = kOffMisc + 16;          // FUSED: A scale of each stage
+    static constexpr uint32_t kOffQRed = kOffScaleA + 4 * STAGES;  // FUSED: amax partials, 2 x 4
+    static constexpr uint32_t kBytes = kOffQRed + 32;
     static constexpr uint32_t kDynamicBytes = kBytes + 1024;
 };
 
@@ -95,11 +117,14 @@ __device__ __forceinline__ void cluster_sync_relaxed() {
     asm volatile("barrier.cluster.arrive.relaxed.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
 }
 
-template <int MP, int STAGES, int NBUF>
-__global__ void __launch_bounds__(kSkinnyThreads, 1)
+template <int MP, int STAGES, int NBUF, bool FUSED>
+__global__ void __launch_bounds__(skinny_threads<FUSED>(), 1)
     skinny_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                        const SkinnyParams p) {
-    using L = SkinnySmem<MP, STAGES, NBUF>;
+    constexpr int kThreads = skinny_threads<FUSED>();
+    constexpr int RA = 4;                  // FUSED: BF16 slabs in flight ahead of the quantizer
+    constexpr int kRing = FUSED ? RA : 0;  // ring slots laid out in shared memory
+    using L = SkinnySmem<MP, STAGES, NBUF, kRing>;
     static_assert(STAGES % 2 == 0 && NBUF % 2 == 0, "each MMA thread must own its stages and buffers");
     constexpr uint32_t kTmemCols = tmem_cols_for(NBUF * MP);
     constexpr uint32_t kIdesc = idesc_e4m3_f32(128, MP);
@@ -111,9 +136,13 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
     uint64_t *tfull = empty + STAGES;
     uint64_t *tempty = tfull + NBUF;
     uint64_t *mdone = tempty + NBUF;
+    uint64_t *afull = mdone + 2;       // FUSED: BF16 slab landed
+    uint64_t *aempty = afull + kRing;  // FUSED: BF16 slab converted
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
     float *red = reinterpret_cast<float *>(smem);  // reuses the stage memory after the K loop
+    float *sa_stage = reinterpret_cast<float *>(smem + L::kOffScaleA);
+    uint32_t *qred = reinterpret_cast<uint32_t *>(smem + L::kOffQRed);
 
     const int warp = static_cast<int>(threadIdx.x >> 5);
     const int lane = lane_id();
@@ -126,14 +155,21 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
 
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+            // FUSED: a stage is full once the weight slab landed and the quantizer
+            // warps wrote the token slab; it is empty once every epilogue warp has
+            // read the stage's A scale
+            mbar_init(&full[s], FUSED ? 2 : 1);
+            mbar_init(&empty[s], FUSED ? 4 : 1);
         }
         for (int b = 0; b < NBUF; ++b) {
             mbar_init(&tfull[b], 1);
             mbar_init(&tempty[b], 4);
         }
         for (int q = 0; q < 2; ++q) mbar_init(&mdone[q], 1);
+        for (int r = 0; r < kRing; ++r) {
+            mbar_init(&afull[r], 1);
+            mbar_init(&aempty[r], 1);
+        }
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmW);
@@ -154,15 +190,15 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
         for (int i = 0; i < nkb; ++i) {
             const int s = i % STAGES;
             const uint32_t u = static_cast<uint32_t>(i / STAGES);
+            const int kb = kb0 + i;
             if (!mbar_wait(&empty[s], (u & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
                 record_failure(p.status, kStatusTimeout, 10, i);
                 *abort_flag = 1;
                 break;
             }
-            const int kb = kb0 + i;
-            mbar_arrive_expect_tx(&full[s], L::kWBytes + L::kXBytes);
+            mbar_arrive_expect_tx(&full[s], FUSED ? L::kWBytes : L::kWBytes + L::kXBytes);
             tma_load_2d(smem + L::kOffW + s * L::kWBytes, &tmW, &full[s], kb * 128, nb * 128);
-            tma_load_2d(smem + L::kOffX + s * L::kXBytes, &tmX, &full[s], kb * 128, 0);
+            if (!FUSED) tma_load_2d(smem + L::kOffX + s * L::kXBytes, &tmX, &full[s], kb * 128, 0);
             issued |= 1u << s;
             parity_bits = (parity_bits & ~(1u << s)) | ((u & 1u) << s);
         }
@@ -171,6 +207,29 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
             if (issued & (1u << s))
                 if (!mbar_wait(&full[s], (parity_bits >> s) & 1u, &never, p.timeout_ns))
                     record_failure(p.status, kStatusTimeout, 10, -1 - s);
+    } else if (FUSED && warp == 3 && lane == 0) {
+        // ------------------------------------ BF16 slab producer (FUSED)
+        // Its own thread, so that the weight stream never waits for the quantizer:
+        // slab i goes to ring slot i % RA, RA slabs ahead of the quantizer.
+        int a_issued = 0;
+        for (int i = 0; i < nkb; ++i) {
+            const int ra = i % RA;
+            const uint32_t ua = static_cast<uint32_t>(i / RA);
+            if (!mbar_wait(&aempty[ra], (ua & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
+                record_failure(p.status, kStatusTimeout, 14, i);
+                *abort_flag = 1;
+                break;
+            }
+            mbar_arrive_expect_tx(&afull[ra], L::kABytes);
+            tma_load_2d(smem + L::kOffA + ra * L::kABytes, &tmX, &afull[ra], (kb0 + i) * 128, 0);
+            a_issued = i + 1;
+        }
+        const int never = 0;
+        for (int r = 0; r < RA && r < a_issued; ++r) {  // the last slab of each ring slot
+            const int last = r + ((a_issued - 1 - r) / RA) * RA;
+            if (!mbar_wait(&afull[r], static_cast<uint32_t>(last / RA) & 1u, &never, p.timeout_ns))
+                record_failure(p.status, kStatusTimeout, 14, -1 - r);
+        }
     } else if ((warp == 1 || warp == 2) && lane == 0) {
         // -------------------------------------------------- MMA (two threads)
         // Thread q issues K blocks i with i % 2 == q; with STAGES and NBUF even
@@ -204,7 +263,84 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
             umma_commit(&mdone[q]);
             if (!mbar_wait(&mdone[q], 0, &never, p.timeout_ns)) record_failure(p.status, kStatusTimeout, 11, -1);
         }
-    } else if (warp >= 4) {
+    } else if (FUSED && warp >= 8) {
+        // ------------------------------------------ activation quantizer (FUSED)
+        // Per K block, all 128 threads: read the BF16 slab from its ring slot
+        // (MP/16 items of one row x 16 columns per thread), reduce amax over the
+        // block, and write the codes into the stage in the swizzled K-major layout
+        // TMA would produce: row r's 16-byte group j at byte r*128 + ((j ^ (r % 8)) * 16).
+        const int qt = static_cast<int>(threadIdx.x) - 256;
+        const int qw = qt >> 5;
+        constexpr int kItems = MP / 16;
+        volatile int *stage_ok = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 8);
+        for (int i = 0; i < nkb; ++i) {
+            const int s = i % STAGES;
+            const uint32_t u = static_cast<uint32_t>(i / STAGES);
+            const int ra = i % RA;
+            const uint32_t ua = static_cast<uint32_t>(i / RA);
+            // one thread waits for the slab and the stage and publishes the outcome,
+            // so that all 128 threads take the same path through the named barriers
+            if (qt == 0)
+                *stage_ok = (mbar_wait(&afull[ra], ua & 1u, abort_flag, p.timeout_ns) &&
+                             mbar_wait(&empty[s], (u & 1u) ^ 1u, abort_flag, p.timeout_ns))
+                                ? 1
+                                : 0;
+            bar_named_sync(2, 128);
+            if (!*stage_ok) {
+                if (qt == 0) {
+                    record_failure(p.status, kStatusTimeout, 13, i);
+                    *abort_flag = 1;
+                }
+                break;
+            }
+            // complete already (slot i % RA cannot refill before this slab is
+            // released): each reader acquires the TMA writes itself
+            mbar_wait(&afull[ra], ua & 1u, abort_flag, p.timeout_ns);
+            const uint8_t *slab = smem + L::kOffA + ra * L::kABytes;
+            const int64_t colbase = static_cast<int64_t>(kb0 + i) * 128;
+            uint4 v[kItems][2];
+            uint32_t m2 = 0;
+#pragma unroll
+            for (int t = 0; t < kItems; ++t) {
+                const int item = qt + t * 128;  // row item / 8, 16-column group item % 8
+                const uint4 *src = reinterpret_cast<const uint4 *>(slab + (item >> 3) * 256 + (item & 7) * 32);
+                v[t][0] = src[0];  // rows past M and columns past K arrive zero-filled
+                v[t][1] = src[1];
+                m2 = amax_fold8(amax_fold8(m2, v[t][0]), v[t][1]);
+            }
+            uint32_t ab = amax_bits_of(m2);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) ab = max(ab, __shfl_xor_sync(0xFFFFFFFFu, ab, o));
+            uint32_t *qr = qred + (i & 1) * 4;  // alternating halves: the previous round may still be read
+            if (lane == 0) qr[qw] = ab;
+            bar_named_sync(2, 128);
+            const BlockScale bs = block_scale(max(max(qr[0], qr[1]), max(qr[2], qr[3])));
+            uint8_t *xs = smem + L::kOffX + s * L::kXBytes;
+#pragma unroll
+            for (int t = 0; t < kItems; ++t) {
+                const int item = qt + t * 128;
+                const int r = item >> 3, j = item & 7;
+                const int64_t col = colbase + j * 16;
+                uint4 codes = make_uint4(0, 0, 0, 0);  // padding quantizes to +0
+                if (r < p.M && col < p.K) {             // K % 16 == 0: a group is whole or absent
+                    const uint2 lo = quantize8(v[t][0], bs), hi = quantize8(v[t][1], bs);
+                    codes = make_uint4(lo.x, lo.y, hi.x, hi.y);
+                    if (nb == 0) *reinterpret_cast<uint4 *>(p.qa_out + static_cast<int64_t>(r) * p.K + col) = codes;
+                }
+                *reinterpret_cast<uint4 *>(xs + r * 128 + ((j ^ (r & 7)) << 4)) = codes;
+            }
+            if (qt == 0) {
+                sa_stage[s] = bs.s;
+                if (nb == 0) p.sa_out[kb0 + i] = bs.s;
+            }
+            fence_async_smem();  // the codes are read by the tensor cores (async proxy)
+            bar_named_sync(2, 128);
+            if (qt == 0) {
+                mbar_arrive(&full[s]);
+                mbar_arrive(&aempty[ra]);
+            }
+        }
+    } else if (warp >= 4 && warp < 8) {
         // -------------------------------------------------------------- epilogue
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;  // output column n = nb*128 + row
@@ -217,8 +353,7 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
             const int buf = i % NBUF;
             const uint32_t v = static_cast<uint32_t>(i / NBUF);
             const int kb = kb0 + i;
-            const float scale = scales.scale(kb, i);
-            const float2 s2 = make_float2(scale, scale);
+            float scale = scales.scale(kb, i);
             if (!mbar_wait(&tfull[buf], v & 1u, abort_flag, p.timeout_ns)) {
                 record_failure(p.status, kStatusTimeout, 12, i);
                 *abort_flag = 1;
@@ -226,7 +361,22 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
             }
             tc_fence_after();
             // the MMAs of this K block are done: its stage may be refilled
-            if (quarter == 0 && lane == 0) mbar_arrive(&empty[i % STAGES]);
+            if (FUSED) {
+                // the stage's A scale, published with the stage's full phase (which
+                // is complete, and cannot advance before this warp's empty arrival)
+                const int s = i % STAGES;
+                if (!mbar_wait(&full[s], static_cast<uint32_t>(i / STAGES) & 1u, abort_flag, p.timeout_ns)) {
+                    record_failure(p.status, kStatusTimeout, 12, i);
+                    *abort_flag = 1;
+                    break;
+                }
+                scale = scale * sa_stage[s];  // = fl32(sA * sB), as in the unfused path
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[s]);
+            } else if (quarter == 0 && lane == 0) {
+                mbar_arrive(&empty[i % STAGES]);
+            }
+            const float2 s2 = make_float2(scale, scale);
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                    static_cast<uint32_t>(buf * MP);
             constexpr int kChunks = MP / 16;
@@ -270,7 +420,7 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
         const int groups = W / 4;         // 4 columns per item
         const int items = p.M * groups;
         const uint32_t red0 = smem_u32(red);
-        for (int it = static_cast<int>(threadIdx.x); it < items; it += kSkinnyThreads) {
+        for (int it = static_cast<int>(threadIdx.x); it < items; it += kThreads) {
             const int m = it / groups;
             const int nl = rank * W + (it - m * groups) * 4;
             const uint32_t off = static_cast<uint32_t>((m * 128 + nl) * 4);
@@ -304,18 +454,26 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
     }
 }
 
-template <int MP, int STAGES, int NBUF>
-static dg_status_t launch_skinny_impl(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream) {
-    using L = SkinnySmem<MP, STAGES, NBUF>;
+template <int MP, int STAGES, int NBUF, bool FUSED>
+static dg_status_t launch_skinny_impl(const GemmArgs &a, const uint16_t *Xa, uint8_t *qa_out, float *sa_out,
+                                      const DeviceInfo &dev, cudaStream_t stream) {
+    using L = SkinnySmem<MP, STAGES, NBUF, FUSED ? 4 : 0>;
     static_assert(L::kDynamicBytes <= 232448, "shared memory budget");
     CUtensorMap tmW, tmX;
     dg_status_t st = make_tmap_2d(&tmW, a.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.N, a.K, 128, 128,
                                   CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != DG_OK) return st;
-    st = make_tmap_2d(&tmX, a.A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.M, a.K, MP, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-    if (st != DG_OK) return st;
+    if (FUSED) {
+        // BF16 slabs of A: MP rows x 128 columns (256 bytes), unswizzled
+        st = make_tmap_2d(&tmX, Xa, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.M, a.K, MP, 128,
+                          CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (st != DG_OK) return st;
+    } else {
+        st = make_tmap_2d(&tmX, a.A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.M, a.K, MP, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (st != DG_OK) return st;
+    }
 
-    auto kernel = skinny_gemm_kernel<MP, STAGES, NBUF>;
+    auto kernel = skinny_gemm_kernel<MP, STAGES, NBUF, FUSED>;
     static thread_local int configured_device = -1;
     int device = 0;
     cudaGetDevice(&device);
@@ -334,7 +492,7 @@ static dg_status_t launch_skinny_impl(const GemmArgs &a, const DeviceInfo &dev, 
     while (S < 8 && 2 * S <= Kb && static_cast<int64_t>(Nt) * 2 * S <= dev.num_sms) S *= 2;
 
     SkinnyParams p;
-    p.sA = a.sA;
+    p.sA = FUSED ? nullptr : a.sA;
     p.sB = a.sB;
     p.C = static_cast<__nv_bfloat16 *>(a.C);
     p.M = static_cast<int>(a.M);
@@ -343,10 +501,14 @@ static dg_status_t launch_skinny_impl(const GemmArgs &a, const DeviceInfo &dev, 
     p.splits = S;
     p.timeout_ns = kernel_control().timeout_ns;
     p.status = kernel_control().status;
+    p.Xa = Xa;
+    p.K = static_cast<int>(a.K);
+    p.qa_out = qa_out;
+    p.sa_out = sa_out;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(Nt * S), 1, 1);
-    cfg.blockDim = dim3(kSkinnyThreads, 1, 1);
+    cfg.blockDim = dim3(static_cast<unsigned>(skinny_threads<FUSED>()), 1, 1);
     cfg.dynamicSmemBytes = L::kDynamicBytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -361,10 +523,18 @@ static dg_status_t launch_skinny_impl(const GemmArgs &a, const DeviceInfo &dev, 
 }
 
 dg_status_t launch_skinny_gemm(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream) {
-    if (a.M <= 16) return launch_skinny_impl<16, 8, 8>(a, dev, stream);
-    if (a.M <= 32) return launch_skinny_impl<32, 8, 8>(a, dev, stream);
-    if (a.M <= 64) return launch_skinny_impl<64, 8, 8>(a, dev, stream);
-    return launch_skinny_impl<128, 6, 4>(a, dev, stream);
+    if (a.M <= 16) return launch_skinny_impl<16, 8, 8, false>(a, nullptr, nullptr, nullptr, dev, stream);
+    if (a.M <= 32) return launch_skinny_impl<32, 8, 8, false>(a, nullptr, nullptr, nullptr, dev, stream);
+    if (a.M <= 64) return launch_skinny_impl<64, 8, 8, false>(a, nullptr, nullptr, nullptr, dev, stream);
+    return launch_skinny_impl<128, 6, 4, false>(a, nullptr, nullptr, nullptr, dev, stream);
+}
+
+dg_status_t launch_skinny_gemm_fused(const GemmArgs &a, const void *A_bf16, uint8_t *qa_out, float *sa_out,
+                                     const DeviceInfo &dev, cudaStream_t stream) {
+    const uint16_t *x = static_cast<const uint16_t *>(A_bf16);
+    if (a.M <= 16) return launch_skinny_impl<16, 8, 8, true>(a, x, qa_out, sa_out, dev, stream);
+    if (a.M <= kFusedMaxM) return launch_skinny_impl<32, 8, 8, true>(a, x, qa_out, sa_out, dev, stream);
+    return DG_ERR_SHAPE;
 }
 
 }  // namespace dg

@@ -98,6 +98,28 @@ dg_status_t dg_fp8_gemm_blockscaled(const uint8_t *A, const float *sA,
                                     int64_t M, int64_t N, int64_t K, cudaStream_t stream);
 
 /*
+ * Block-scaled GEMM from BF16 activations: A is quantized per 128x128 block
+ * exactly as dg_quantize_blockwise does (same codes, same scales, bit for bit),
+ * then C = A * B^T as in dg_fp8_gemm_blockscaled.  Activation scales are
+ * recomputed on every call while weight scales are computed once
+ * (2kiu.com/news/5461879 §5), so this is the call a layer makes per step.
+ *
+ * A_bf16 : [M][K] BF16, 16-byte aligned.
+ * B, sB  : as in dg_fp8_gemm_blockscaled (quantized once, e.g. by dg_quantize_blockwise).
+ * C      : [M][N] BF16 out, 16-byte aligned.
+ * QA     : [M][K] E4M3 out, 16-byte aligned; sA : [ceil(M/128)][ceil(K/128)] FP32 out.
+ *          Caller-owned: they receive A's codes and scales (the library allocates
+ *          nothing).
+ * Shapes as in dg_fp8_gemm_blockscaled (N % 16 == 0, K % 16 == 0, K > 0).
+ * M <= 32: one launch -- the skinny kernel quantizes A inside its producer
+ * stage (no separate pass over A).  Larger M: the block quantizer, then the
+ * FP8 GEMM, on `stream`.  M == 0 or N == 0 is a no-op.
+ */
+dg_status_t dg_fp8_gemm_blockscaled_bf16a(const void *A_bf16, const uint8_t *B, const float *sB,
+                                          void *C_bf16, uint8_t *QA, float *sA,
+                                          int64_t M, int64_t N, int64_t K, cudaStream_t stream);
+
+/*
  * MoE grouped-contiguous block-scaled GEMM (nxmr.cn/news/132300 §2.2;
  * 2kiu.com/news/5461879 §2.2): expert g owns rows [off[g], off[g+1]) of A and
  * C, every off[g] a multiple of 128, and for those rows

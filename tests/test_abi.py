@@ -63,5 +63,10 @@ def test_host_validation_without_device(lib):
     assert lib.dg_fp8_grouped_gemm_contiguous(null, null, null, null, null, null, 128, 2, 64, 128, null) == 2
     assert lib.dg_fp8_grouped_gemm_contiguous(null, null, null, null, null, null, 0, 2, 128, 128, null) == 0
     assert lib.dg_fp8_grouped_gemm_contiguous(null, null, null, null, null, null, 128, 2, 128, 128, null) == 1
+    # the BF16-activation GEMM: shapes first, then pointers
+    assert lib.dg_fp8_gemm_blockscaled_bf16a(null, null, null, null, null, null, 8, 16, 100, null) == 2
+    assert lib.dg_fp8_gemm_blockscaled_bf16a(null, null, null, null, null, null, 8, 24, 128, null) == 2
+    assert lib.dg_fp8_gemm_blockscaled_bf16a(null, null, null, null, null, null, 0, 16, 128, null) == 0
+    assert lib.dg_fp8_gemm_blockscaled_bf16a(null, null, null, null, null, null, 8, 16, 128, null) == 1
     odd = ctypes.c_void_p(0x1001)
     assert lib.dg_fp8_gemm_blockscaled(odd, odd, odd, odd, odd, 8, 16, 128, null) == 3
