@@ -14,6 +14,8 @@ Recipe (every draw is CPU-side and seeded, so any machine reproduces it):
     permuted) and then the per-expert token-slot counts from a multinomial.
   * Grouped layout: each expert's rows padded up to a multiple of 128; padding
     rows of A are zero; group_offsets is the int32 prefix sum of padded counts.
+  * Masked layout: expert g's tokens are rows 0..count_g-1 of its M_max-row slab;
+    the rows after them hold N(0, 100^2) junk, which no output may depend on.
 """
 from __future__ import annotations
 
@@ -175,6 +177,40 @@ def grouped_custom(G: int, N: int, K: int, counts, seed: int) -> Grouped:
             a[off[g]:off[g] + c] = torch.randn((c, K), generator=ga).to(torch.bfloat16)
     b = bf16_normal((G, N, K), 0.02, seed + 500_000)
     return Grouped(f"grouped_g{G}_n{N}_k{K}", G, N, K, counts, off, a, b, seed)
+
+
+@dataclass
+class Masked:
+    name: str
+    G: int
+    M_max: int
+    N: int
+    K: int
+    counts: np.ndarray   # int64 [G], tokens per expert
+    A: torch.Tensor      # BF16 [G][M_max][K]; rows >= counts[g] are junk
+    B: torch.Tensor      # BF16 [G][N][K]
+    seed: int
+
+
+def masked_custom(G: int, M_max: int, N: int, K: int, counts, seed: int) -> Masked:
+    """Masked MoE layout with the given per-expert counts (0..M_max)."""
+    counts = np.asarray(counts, dtype=np.int64)
+    ga = torch.Generator().manual_seed(seed)
+    a = torch.randn((G, M_max, K), generator=ga, dtype=torch.float32)
+    for g in range(G):
+        a[g, int(counts[g]):] *= 100.0
+    b = bf16_normal((G, N, K), 0.02, seed + 500_000)
+    return Masked(f"masked_g{G}_m{M_max}_n{N}_k{K}", G, M_max, N, K, counts, a.to(torch.bfloat16), b, seed)
+
+
+def moe_masked_g8() -> Masked:
+    """The moe_g8 routing (8 experts, N=K=4096, 16384 slots, Dirichlet(1)) in the
+    masked layout: slabs of M_max = the largest count rounded up to 128."""
+    counts = moe_counts(8, 16384, 1004, "dirichlet")
+    m_max = int((counts.max() + ALIGN_M - 1) // ALIGN_M * ALIGN_M)
+    m = masked_custom(8, m_max, 4096, 4096, counts, 1007)
+    m.name = "moe_masked_g8_n4096_k4096"
+    return m
 
 
 def bf16_bits(t: torch.Tensor) -> np.ndarray:

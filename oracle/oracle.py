@@ -175,6 +175,26 @@ def grouped_gemm_ref(A, sA, B, sB, offsets, rows, cols=None) -> np.ndarray:
     return out
 
 
+def masked_gemm_ref(A, sA, B, sB, masked_m, cols=None) -> np.ndarray:
+    """FP64 block formula for the masked MoE layout: expert g's first masked_m[g] rows.
+
+    A [G][M_max][K] codes, sA [G][ceil(M_max/128)][ceil(K/128)], B [G][N][K],
+    sB [G][ceil(N/128)][ceil(K/128)], masked_m [G] (clamped to [0, M_max]).  Each
+    expert is the dense formula on its own slab (2kiu.com/news/5461879 §2.2: only M
+    varies between experts).  Rows at or past masked_m[g] come back as NaN.
+    """
+    A = np.ascontiguousarray(A, dtype=np.uint8)
+    G, Mmax, K = A.shape
+    N = B.shape[1]
+    nc = N if cols is None else len(cols)
+    out = np.full((G, Mmax, nc), np.nan, dtype=np.float64)
+    for g in range(G):
+        m = min(max(int(masked_m[g]), 0), Mmax)
+        if m:
+            out[g, :m] = gemm_ref(A[g], sA[g], B[g], sB[g], rows=np.arange(m), cols=cols)
+    return out
+
+
 # ----------------------------------------------------------------------- checking
 RTOL = 1e-2
 ATOL_RMS = 1e-3

@@ -436,3 +436,35 @@ def test_gemm_ref_k_tail_equals_zero_padded_full_blocks(K):
     tail = oracle.gemm_ref(A, sA2, B, sB) - oracle.gemm_ref(head, sA2, B, sB)
     tail1 = ref - oracle.gemm_ref(head, sA, B, sB)
     assert np.allclose(tail, 2 * tail1, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+
+
+def test_masked_ref_equals_contiguous_ref_on_packed_rows():
+    """The masked layout and the grouped-contiguous layout hold the same tokens: the
+    masked formula must give the contiguous routine's values bit for bit (two routines
+    with different expert lookups), NaN past each count, and clamp counts to M_max."""
+    rng = np.random.default_rng(31)
+    G, Mmax, N, K = 4, 200, 144, 256
+    counts = np.array([0, 200, 77, 129])
+    A = random_finite_codes(rng, (G, Mmax, K))
+    sA = random_scales(rng, (G, 2, 2))
+    B = random_finite_codes(rng, (G, N, K))
+    sB = random_scales(rng, (G, 2, 2))
+    got = oracle.masked_gemm_ref(A, sA, B, sB, counts)
+    # packed contiguous layout: expert g's rows at a 128-aligned offset, same m-block scales
+    padded = (counts + 127) // 128 * 128
+    off = np.concatenate([[0], np.cumsum(padded)]).astype(np.int32)
+    Ac = np.zeros((int(off[-1]), K), np.uint8)
+    sAc = np.ones((int(off[-1]) // 128, 2), np.float32)
+    for g in range(G):
+        Ac[off[g]:off[g] + counts[g]] = A[g, :counts[g]]
+        nb = padded[g] // 128
+        sAc[off[g] // 128:off[g] // 128 + nb] = sA[g, :nb]
+    rows = np.concatenate([np.arange(off[g], off[g] + counts[g]) for g in range(G)]).astype(np.int64)
+    want = oracle.grouped_gemm_ref(Ac, sAc, B, sB, off, rows)
+    got_rows = np.concatenate([got[g, :counts[g]] for g in range(G)])
+    assert np.array_equal(got_rows, want)
+    for g in range(G):
+        assert np.all(np.isnan(got[g, counts[g]:]))
+    # clamping: a count past M_max acts as M_max, a negative one as 0
+    clamped = oracle.masked_gemm_ref(A, sA, B, sB, np.array([-5, 999, 77, 129]))
+    assert np.array_equal(clamped[1], got[1]) and np.all(np.isnan(clamped[0]))
