@@ -74,7 +74,7 @@ def load_peaks():
 
 # ------------------------------------------------------------------ workloads
 WORKLOADS = ("dense_4096_outliers", "dense_512", "dense_8192", "skinny_m1", "skinny_m16", "skinny_m64",
-             "skinny_m128", "moe_g8", "moe_g64_zipf")
+             "skinny_m128", "moe_g8", "moe_g64_zipf", "moe_masked_g8")
 
 
 def make_workload(name):
@@ -91,12 +91,25 @@ def make_workload(name):
         return inputs.moe_g8()
     if name == "moe_g64_zipf":
         return inputs.moe_g64_zipf()
+    if name == "moe_masked_g8":
+        return inputs.moe_masked_g8()
     raise SystemExit(f"unknown workload {name}")
 
 
 def workload_facts(w):
     """(flops per step on real tokens, algorithmic GEMM bytes, rows of A, config dict)."""
-    from fp8_block_scaled_scales_b200.inputs import Grouped
+    from fp8_block_scaled_scales_b200.inputs import Grouped, Masked
+    if isinstance(w, Masked):
+        real = int(w.counts.sum())
+        flops = 2.0 * real * w.N * w.K
+        kb = -(-w.K // 128)
+        mblocks = int(((w.counts + 127) // 128).sum())
+        # the m-blocks that hold tokens are read and written; B and its scales once
+        gemm_bytes = (mblocks * 128 * (w.K + 2 * w.N) + w.G * w.N * w.K
+                      + 4 * (mblocks + w.G * (w.N // 128)) * kb)
+        cfg = {"workload": w.name, "experts": w.G, "N": w.N, "K": w.K, "token_slots": real,
+               "m_max": w.M_max, "layout": "masked (counts read on the device)"}
+        return flops, gemm_bytes, w.G * w.M_max, cfg
     if isinstance(w, Grouped):
         real = int(w.counts.sum())
         flops = 2.0 * real * w.N * w.K
@@ -178,7 +191,21 @@ def oracle_sample(w, rows_sample: int, seed: int = 0):
     (cached weights), matching the GPU step."""
     import oracle
     from fp8_block_scaled_scales_b200 import inputs
-    from fp8_block_scaled_scales_b200.inputs import Grouped
+    from fp8_block_scaled_scales_b200.inputs import Grouped, Masked
+    if isinstance(w, Masked):
+        # the expert with the most tokens: its first rows_sample tokens (whole 128-row blocks)
+        g = int(np.argmax(w.counts))
+        qb, sb = oracle.quantize_blockwise(inputs.bf16_bits(w.B[g]))
+        rows = int(min(int(w.counts[g]), max(1, rows_sample // 128) * 128))
+        nblk = -(-rows // 128)
+        t0 = time.perf_counter()
+        qa, sa = oracle.quantize_blockwise(inputs.bf16_bits(w.A[g, :nblk * 128]))
+        ref = oracle.gemm_ref(qa, sa, qb, sb, rows=np.arange(rows))
+        out = oracle.bf16_from_double(ref)
+        dt = time.perf_counter() - t0
+        del out
+        desc = f"{rows} token rows of expert {g} x all {w.N} columns, K={w.K}, their A quantization included"
+        return dt, 2.0 * rows * w.N * w.K, oracle.num_threads(), desc
     if isinstance(w, Grouped):
         qb = np.stack([oracle.quantize_blockwise(inputs.bf16_bits(w.B[g]))[0] for g in range(w.G)])
         sb = np.stack([oracle.quantize_blockwise(inputs.bf16_bits(w.B[g]))[1] for g in range(w.G)])
@@ -213,8 +240,8 @@ def oracle_sample(w, rows_sample: int, seed: int = 0):
 
 
 def default_oracle_rows(w) -> int:
-    from fp8_block_scaled_scales_b200.inputs import Grouped
-    if isinstance(w, Grouped):
+    from fp8_block_scaled_scales_b200.inputs import Grouped, Masked
+    if isinstance(w, (Grouped, Masked)):
         return 1024
     per_row = w.N * w.K
     return int(max(1, min(w.M, 1.2e11 // per_row)))
@@ -255,32 +282,40 @@ def max_over_ranks(x: float, world: int) -> float:
 # -------------------------------------------------------------- dg impl
 def run_dg(args):
     from fp8_block_scaled_scales_b200 import binding
-    from fp8_block_scaled_scales_b200.inputs import Grouped
+    from fp8_block_scaled_scales_b200.inputs import Grouped, Masked
 
     world, rank, local = dist_setup(args.gpus)
     w = make_workload(args.workload)
     flops, gemm_bytes, rows_a, cfg = workload_facts(w)
     grouped = isinstance(w, Grouped)
-    skinny = (not grouped) and w.M <= 128
+    masked = isinstance(w, Masked)
+    skinny = not (grouped or masked) and w.M <= 128
     fused = skinny and w.M <= FUSED_MAX_M  # one launch: the GEMM quantizes A itself
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream()
 
-    A_host = w.A.contiguous()
+    A_host = w.A.contiguous().reshape(rows_a, w.K)  # masked: the [G][M_max] slabs as rows
     A = A_host.to(dev)
-    B = w.B.reshape(-1, w.K).to(dev) if grouped else w.B.to(dev)
+    B = w.B.reshape(-1, w.K).to(dev) if (grouped or masked) else w.B.to(dev)
     qb, sb = binding.quantize_blockwise(B)                    # cached weights
-    if grouped:
+    if grouped or masked:
         qb = qb.view(w.G, w.N, w.K)
-        sb = sb.view(w.G, w.N // 128, w.K // 128)
+        sb = sb.view(w.G, w.N // 128, -(-w.K // 128))
+    if grouped:
         off = torch.from_numpy(w.offsets).to(dev)
+    if masked:
+        assert w.M_max % 128 == 0  # slab blocks coincide with the row blocks quantized below
+        mm = torch.from_numpy(w.counts.astype(np.int32)).to(dev)
     qa = torch.empty((rows_a, w.K), dtype=torch.uint8, device=dev)
     sa = torch.empty((-(-rows_a // 128), -(-w.K // 128)), dtype=torch.float32, device=dev)
     C = torch.empty((rows_a, w.N), dtype=torch.bfloat16, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
 
     def gemm():
-        if grouped:
+        if masked:
+            binding.grouped_gemm_masked(qa.view(w.G, w.M_max, w.K), sa.view(w.G, w.M_max // 128, -1), qb, sb, mm,
+                                        C=C.view(w.G, w.M_max, w.N))
+        elif grouped:
             binding.grouped_gemm_contiguous(qa, sa, qb, sb, off, C=C)
         else:
             binding.gemm_blockscaled(qa, sa, qb, sb, C=C)
@@ -382,7 +417,7 @@ def run_dg(args):
                 "frac": round(achieved / peak, 4)}
     roof["peak_source"] = (f"{peaks['source']}: bf16 cuBLAS burst {peaks['bf16_tflops']} TF/s x {FP8_OVER_BF16}"
                            if roof["bound"] == "tensor" else f"{peaks['source']}: HBM copy {peaks['hbm_gbs']} GB/s")
-    kfile = "gemm_pair.cu" if not (grouped or skinny) else ("gemm_tile.cu" if grouped else "gemm_skinny.cu")
+    kfile = ("gemm_tile.cu" if (grouped or masked) else "gemm_skinny.cu" if skinny else "gemm_pair.cu")
     roof["traffic"] = ncu_traffic(args.workload, kfile)
     roof["algorithmic_bytes"] = int(gemm_bytes)
     roof["kernel_ms"] = round(ms_gemm, 5)

@@ -5,5 +5,5 @@ include/dg.h); this package is its Python binding plus the seeded input
 generators used by the tests and the benchmark.
 """
 from .binding import (DGError, gemm_blockscaled, gemm_blockscaled_bf16a,  # noqa: F401
-                      grouped_gemm_contiguous, last_device_status, quantize_blockwise,
+                      grouped_gemm_contiguous, grouped_gemm_masked, last_device_status, quantize_blockwise,
                       set_kernel_control, version)

@@ -23,7 +23,7 @@ KERNELS = {"auto": 0, "tile": 1, "skinny": 2, "pair": 3}
 
 # every symbol include/dg.h declares
 EXPORTS = ("dg_quantize_blockwise", "dg_fp8_gemm_blockscaled", "dg_fp8_gemm_blockscaled_bf16a",
-           "dg_fp8_grouped_gemm_contiguous",
+           "dg_fp8_grouped_gemm_contiguous", "dg_fp8_grouped_gemm_masked",
            "dg_fp8_gemm_blockscaled_select", "dg_status_string", "dg_get_last_device_status",
            "dg_version", "dg_test_set_kernel_control")
 
@@ -52,9 +52,10 @@ def lib() -> ctypes.CDLL:
     L.dg_fp8_gemm_blockscaled_select.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, vp]
     L.dg_fp8_gemm_blockscaled_bf16a.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp]
     L.dg_fp8_grouped_gemm_contiguous.argtypes = [vp, vp, vp, vp, vp, vp, i64, i32, i64, i64, vp]
+    L.dg_fp8_grouped_gemm_masked.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, i64, i64, vp]
     for f in ("dg_quantize_blockwise", "dg_fp8_gemm_blockscaled", "dg_fp8_gemm_blockscaled_select",
               "dg_fp8_gemm_blockscaled_bf16a",
-              "dg_fp8_grouped_gemm_contiguous", "dg_get_last_device_status"):
+              "dg_fp8_grouped_gemm_contiguous", "dg_fp8_grouped_gemm_masked", "dg_get_last_device_status"):
         getattr(L, f).restype = ctypes.c_int
     L.dg_get_last_device_status.argtypes = [vp]
     L.dg_status_string.restype = ctypes.c_char_p
@@ -150,6 +151,21 @@ def grouped_gemm_contiguous(A, sA, B, sB, offsets, C=None, stream=None):
     _check(lib().dg_fp8_grouped_gemm_contiguous(_p(A), _p(sA), _p(B), _p(sB), _p(C), _p(offsets), Mcap, G,
                                                 N, K, _stream(stream)),
            "dg_fp8_grouped_gemm_contiguous")
+    return C
+
+
+def grouped_gemm_masked(A, sA, B, sB, masked_m, C=None, stream=None):
+    """Masked MoE GEMM: A [G][M_max][K], B [G][N][K], masked_m int32 [G] (device).
+
+    Rows at or past masked_m[g] of C are not written (a new C is zero-filled)."""
+    A, B = _u8(A), _u8(B)
+    G, Mmax, K = A.shape
+    N = B.shape[1]
+    if C is None:
+        C = torch.zeros((G, Mmax, N), dtype=torch.bfloat16, device=A.device)
+    _check(lib().dg_fp8_grouped_gemm_masked(_p(A), _p(sA), _p(B), _p(sB), _p(C), _p(masked_m), G, Mmax, N, K,
+                                            _stream(stream)),
+           "dg_fp8_grouped_gemm_masked")
     return C
 
 

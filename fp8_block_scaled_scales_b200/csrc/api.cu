@@ -174,7 +174,7 @@ dg_status_t dg_fp8_gemm_blockscaled_select(const uint8_t *A, const float *sA, co
     GemmArgs a = {A, sA, B, sB, C_bf16, nullptr, M, N, K, 0};
     if (kernel == DG_KERNEL_AUTO) kernel = M <= 128 ? DG_KERNEL_SKINNY : DG_KERNEL_PAIR;
     if (kernel == DG_KERNEL_SKINNY) return launch_skinny_gemm(a, dev, stream);
-    if (kernel == DG_KERNEL_TILE) return launch_tile_gemm(a, false, dev, stream);
+    if (kernel == DG_KERNEL_TILE) return launch_tile_gemm(a, 0, dev, stream);
     return N <= 128 ? launch_pair_gemm_n128(a, dev, stream) : launch_pair_gemm(a, dev, stream);
 }
 
@@ -206,6 +206,27 @@ dg_status_t dg_fp8_gemm_blockscaled_bf16a(const void *A_bf16, const uint8_t *B, 
     return dg_fp8_gemm_blockscaled_select(QA, sA, B, sB, C_bf16, M, N, K, DG_KERNEL_AUTO, stream);
 }
 
+dg_status_t dg_fp8_grouped_gemm_masked(const uint8_t *A, const float *sA, const uint8_t *B, const float *sB,
+                                       void *C_bf16, const int32_t *masked_m, int G, int64_t M_max, int64_t N,
+                                       int64_t K, cudaStream_t stream) {
+    if (G < 1 || G > 256 || M_max < 0 || N < 0 || N % 128 != 0 || K <= 0 || K % 16 != 0) return DG_ERR_SHAPE;
+    if (static_cast<int64_t>(G) * M_max > 0x7FFFFFFFLL || static_cast<int64_t>(G) * N > 0x7FFFFFFFLL ||
+        K > 0x7FFFFFFFLL)
+        return DG_ERR_SHAPE;
+    if (M_max == 0 || N == 0) return DG_OK;
+    if (!masked_m) return DG_ERR_INVALID_ARG;
+    if (!aligned(masked_m, 4)) return DG_ERR_ALIGNMENT;
+    dg_status_t st = check_gemm_common(A, sA, B, sB, C_bf16);
+    if (st != DG_OK) return st;
+    DeviceInfo dev;
+    st = current_device(&dev, nullptr);
+    if (st != DG_OK) return st;
+    GemmArgs a = {A, sA, B, sB, C_bf16, nullptr, static_cast<int64_t>(G) * M_max, N, K, G};
+    a.masked_m = masked_m;
+    a.m_max = M_max;
+    return launch_tile_gemm(a, 2, dev, stream);
+}
+
 dg_status_t dg_fp8_grouped_gemm_contiguous(const uint8_t *A, const float *sA, const uint8_t *B, const float *sB,
                                            void *C_bf16, const int32_t *group_offsets, int64_t M_total_capacity,
                                            int G, int64_t N, int64_t K, cudaStream_t stream) {
@@ -223,7 +244,7 @@ dg_status_t dg_fp8_grouped_gemm_contiguous(const uint8_t *A, const float *sA, co
     st = current_device(&dev, nullptr);
     if (st != DG_OK) return st;
     GemmArgs a = {A, sA, B, sB, C_bf16, group_offsets, M_total_capacity, N, K, G};
-    return launch_tile_gemm(a, true, dev, stream);
+    return launch_tile_gemm(a, 1, dev, stream);
 }
 
 }  // extern "C"

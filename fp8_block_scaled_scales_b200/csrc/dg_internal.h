@@ -42,13 +42,16 @@ struct GemmArgs {
     const float *sB;
     void *C;
     const int32_t *offsets;  // grouped only
-    int64_t M;               // dense: M, grouped: M_total_capacity
+    int64_t M;               // dense: M, grouped: M_total_capacity, masked: G * M_max
     int64_t N;
     int64_t K;
     int G;                   // grouped only
+    const int32_t *masked_m = nullptr;  // masked only: tokens per expert (device)
+    int64_t m_max = 0;                  // masked only: rows per expert slab
 };
 
-dg_status_t launch_tile_gemm(const GemmArgs &a, bool grouped, const DeviceInfo &dev, cudaStream_t stream);
+// group: 0 dense, 1 grouped-contiguous, 2 masked
+dg_status_t launch_tile_gemm(const GemmArgs &a, int group, const DeviceInfo &dev, cudaStream_t stream);
 dg_status_t launch_pair_gemm(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream);
 dg_status_t launch_pair_gemm_n128(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream);
 dg_status_t launch_skinny_gemm(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream);

@@ -31,10 +31,15 @@
 // the tensor cores run ahead by NBUF - 1 K blocks; at a tile boundary they run into the
 // next tile while the epilogue writes the previous tile's output.
 //
-// Grouped form: m-blocks run over the padded concatenation of the experts' rows;
-// the expert of m-block i is the g with off[g] <= 128 i < off[g+1] (the pages'
-// "experts stored contiguously by expert id", nxmr.cn/news/132300 §2.2); B is
-// addressed as rows g*N + n of a [G*N][K] matrix.
+// Grouped forms (GMODE): B is addressed as rows g*N + n of a [G*N][K] matrix.
+//   kContiguous: m-blocks run over the padded concatenation of the experts' rows;
+//     the expert of m-block i is the g with off[g] <= 128 i < off[g+1] (the pages'
+//     "experts stored contiguously by expert id", nxmr.cn/news/132300 §2.2).
+//   kMasked: expert g owns a slab of M_max rows of A and C and uses its first
+//     masked_m[g] (a device count; only M varies between experts and it changes
+//     from call to call, 2kiu.com/news/5461879 §2.2).  Each CTA turns the counts
+//     into a prefix of m-blocks in shared memory and walks only the m-blocks that
+//     hold tokens; rows at or past masked_m[g] are never written.
 #include <cuda_bf16.h>
 
 #include "dg_device.cuh"
@@ -42,10 +47,17 @@
 
 namespace dg {
 
+enum GroupMode { kDense = 0, kContiguous = 1, kMasked = 2 };
+constexpr int kMaskedMaxG = 256;  // prefix table in shared memory
+
 struct TileParams {
     const float *sA;
     const float *sB;
-    const int32_t *offsets;
+    const int32_t *offsets;   // kContiguous: off[G+1]
+    const int32_t *masked_m;  // kMasked: tokens per expert
+    int m_max;                // kMasked: rows per expert slab
+    int mb_max;               // kMasked: ceil(m_max / 128), sA rows per expert
+    __nv_bfloat16 *C;         // kMasked: rows stored one by one at an expert's last block
     int G;
     int num_m_cap;    // m-blocks of the allocation (dense: ceil(M/128))
     int num_n_tiles;  // ceil(N / BN)
@@ -88,7 +100,7 @@ __device__ __forceinline__ int expert_of_row(const int32_t *off, int G, int row)
     return lo;
 }
 
-template <int BN, int STAGES, int NBUF>
+template <int BN, int STAGES, int NBUF, int GMODE>
 struct TileSmem {
     static constexpr uint32_t kABytes = 128 * 128;
     static constexpr uint32_t kBBytes = BN * 128;
@@ -99,15 +111,67 @@ struct TileSmem {
     static constexpr uint32_t kOffBar = kOffC + 8 * kCBoxBytes;
     static constexpr uint32_t kNumBars = 2 * STAGES + 2 * NBUF + 2;
     static constexpr uint32_t kOffMisc = kOffBar + 8 * kNumBars;
-    static constexpr uint32_t kBytes = kOffMisc + 16;
+    static constexpr uint32_t kOffPrefix = kOffMisc + 16;  // kMasked: m-block prefix, G + 1 ints
+    static constexpr uint32_t kBytes = kOffPrefix + (GMODE == kMasked ? 4 * (kMaskedMaxG + 4) : 0);
     static constexpr uint32_t kDynamicBytes = kBytes + 1024;  // slack for 1024-byte alignment
 };
 
-template <int BN, bool GROUPED, int STAGES, int NBUF>
+// Where tile t's operands and output live.
+struct TileInfo {
+    int a_row;   // TMA row of A (and C) where the tile's 128 rows start
+    int b_row;   // TMA row of B
+    int sa_row;  // row of sA
+    int sb_row;  // row of sB for the tile's first 128 columns
+    int rows;    // rows of the tile that hold output (kMasked: up to masked_m; else 128)
+};
+
+// Number of m-blocks; kMasked also fills the prefix table (all threads call it
+// after the table is built, so they agree).
+template <int GMODE>
+__device__ __forceinline__ int count_m_blocks(const TileParams &p, const int *prefix) {
+    if (GMODE == kMasked) return prefix[p.G];
+    if (GMODE == kContiguous) return min(p.num_m_cap, __ldg(p.offsets + p.G) / 128);
+    return p.num_m_cap;
+}
+
+__device__ __forceinline__ int masked_count(const TileParams &p, int g) {
+    return min(max(__ldg(p.masked_m + g), 0), p.m_max);  // counts outside [0, M_max] are clamped
+}
+
+template <int BN, int GMODE>
+__device__ __forceinline__ TileInfo resolve_tile(const TileParams &p, const int *prefix, int t, int num_m,
+                                                 int &nb) {
+    int mb;
+    tile_coords(t, num_m, p.num_n_tiles, mb, nb);
+    TileInfo ti;
+    if (GMODE == kMasked) {
+        int lo = 0, hi = p.G;  // the g with prefix[g] <= mb < prefix[g+1]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (prefix[mid] <= mb) lo = mid; else hi = mid;
+        }
+        const int local = mb - prefix[lo];
+        ti.a_row = lo * p.m_max + local * 128;
+        ti.b_row = lo * p.N + nb * BN;
+        ti.sa_row = lo * p.mb_max + local;
+        ti.sb_row = lo * p.Nb;
+        ti.rows = min(128, masked_count(p, lo) - local * 128);
+    } else {
+        const int g = GMODE == kContiguous ? expert_of_row(p.offsets, p.G, mb * 128) : 0;
+        ti.a_row = mb * 128;
+        ti.b_row = g * p.N + nb * BN;
+        ti.sa_row = mb;
+        ti.sb_row = g * p.Nb;
+        ti.rows = 128;
+    }
+    return ti;
+}
+
+template <int BN, int GMODE, int STAGES, int NBUF>
 __global__ void __launch_bounds__(kTileThreads, 1)
     tile_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, const TileParams p) {
-    using L = TileSmem<BN, STAGES, NBUF>;
+    using L = TileSmem<BN, STAGES, NBUF, GMODE>;
         constexpr int kColsPerWarp = BN / 2;
     constexpr uint32_t kTmemCols = tmem_cols_for(NBUF * BN);
     constexpr uint32_t kIdesc = idesc_e4m3_f32(128, BN);
@@ -121,6 +185,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
     uint64_t *mdone = tempty + NBUF;  // one per MMA thread: all its MMAs complete
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
+    int *prefix = reinterpret_cast<int *>(smem + L::kOffPrefix);  // kMasked only
 
     const int warp = static_cast<int>(threadIdx.x >> 5);
     const int lane = lane_id();
@@ -145,12 +210,39 @@ __global__ void __launch_bounds__(kTileThreads, 1)
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
+    if (GMODE == kMasked && warp == 3) {
+        // prefix[g] = sum over h < g of ceil(count_h / 128): lane l takes experts
+        // 8l .. 8l+7, then an exclusive scan of the lane sums
+        constexpr int kPer = kMaskedMaxG / 32;
+        int blocks[kPer];
+        int sum = 0;
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            const int g = lane * kPer + i;
+            blocks[i] = g < p.G ? (masked_count(p, g) + 127) / 128 : 0;
+            sum += blocks[i];
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - sum;
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            const int g = lane * kPer + i;
+            if (g < p.G) prefix[g] = run;
+            run += blocks[i];
+        }
+        if (lane == 31) prefix[p.G] = incl;
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    const int num_m = GROUPED ? min(p.num_m_cap, __ldg(p.offsets + p.G) / 128) : p.num_m_cap;
+    const int num_m = count_m_blocks<GMODE>(p, prefix);
     const int num_tiles = num_m * p.num_n_tiles;
     const int Kb = p.Kb;
 
@@ -162,10 +254,8 @@ __global__ void __launch_bounds__(kTileThreads, 1)
             int it = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-                int mb, nb;
-                tile_coords(t, num_m, p.num_n_tiles, mb, nb);
-                int b_row = nb * BN;
-                if (GROUPED) b_row += expert_of_row(p.offsets, p.G, mb * 128) * p.N;
+                int nb;
+                const TileInfo ti = resolve_tile<BN, GMODE>(p, prefix, t, num_m, nb);
                 for (int kb = 0; kb < Kb; ++kb, ++it) {
                     const int s = it % STAGES;
                     const uint32_t u = static_cast<uint32_t>(it / STAGES);
@@ -177,8 +267,8 @@ __global__ void __launch_bounds__(kTileThreads, 1)
                     }
                     if ((p.debug_flags & 1) && it == 0) continue;  // test hook: never fill stage 0
                     mbar_arrive_expect_tx(&full[s], L::kABytes + L::kBBytes);
-                    tma_load_2d(smem + L::kOffA + s * L::kABytes, &tmA, &full[s], kb * 128, mb * 128);
-                    tma_load_2d(smem + L::kOffB + s * L::kBBytes, &tmB, &full[s], kb * 128, b_row);
+                    tma_load_2d(smem + L::kOffA + s * L::kABytes, &tmA, &full[s], kb * 128, ti.a_row);
+                    tma_load_2d(smem + L::kOffB + s * L::kBBytes, &tmB, &full[s], kb * 128, ti.b_row);
                     issued |= 1u << s;
                     parity_bits = (parity_bits & ~(1u << s)) | ((u & 1u) << s);
                 }
@@ -246,15 +336,14 @@ __global__ void __launch_bounds__(kTileThreads, 1)
         int kc = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-            int mb, nb;
-            tile_coords(t, num_m, p.num_n_tiles, mb, nb);
+            int nb;
+            const TileInfo ti = resolve_tile<BN, GMODE>(p, prefix, t, num_m, nb);
             const int col0 = nb * BN + half * kColsPerWarp;
             const int nb128 = col0 / 128;
             const bool n_valid = nb128 < p.Nb;
-            int sb_row = nb128;
-            if (GROUPED) sb_row += expert_of_row(p.offsets, p.G, mb * 128) * p.Nb;
+            const int sb_row = ti.sb_row + nb128;
             ScaleStream scales;
-            scales.start(p.sA + static_cast<int64_t>(mb) * Kb, p.sB + static_cast<int64_t>(sb_row) * Kb, 0,
+            scales.start(p.sA + static_cast<int64_t>(ti.sa_row) * Kb, p.sB + static_cast<int64_t>(sb_row) * Kb, 0,
                          n_valid ? Kb : 0);
 #pragma unroll
             for (int i = 0; i < kColsPerWarp / 2; ++i) acc[i] = make_float2(0.0f, 0.0f);
@@ -299,10 +388,25 @@ __global__ void __launch_bounds__(kTileThreads, 1)
                 }
             }
             if (!ok) break;
-            // BF16 output: rows mb*128 + 32*quarter + lane, columns col0 .. col0 + kColsPerWarp
-            const int row0 = mb * 128 + quarter * 32;
+            // BF16 output: rows a_row + 32*quarter + lane, columns col0 .. col0 + kColsPerWarp
+            const int row0 = ti.a_row + quarter * 32;
+            const int vrows = ti.rows - quarter * 32;  // rows of this warp's box that hold output
 #pragma unroll
             for (int j = 0; j < kColsPerWarp / 64; ++j) {
+                if (GMODE == kMasked && vrows < 32) {
+                    // the box runs past the expert's tokens: each row that holds
+                    // output stores itself, the rest of the slab is left untouched
+                    if (lane < vrows && col0 + j * 64 < p.N) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(p.C + static_cast<int64_t>(row0 + lane) * p.N + col0 + j * 64);
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            const float2 *x = acc + j * 32 + c * 4;
+                            dst[c] = make_uint4(pack_bf16x2(x[0].x, x[0].y), pack_bf16x2(x[1].x, x[1].y),
+                                                pack_bf16x2(x[2].x, x[2].y), pack_bf16x2(x[3].x, x[3].y));
+                        }
+                    }
+                    continue;
+                }
                 if (lane == 0) bulk_wait_read0();  // the previous store has finished reading cstage
                 __syncwarp();
                 uint8_t *rowp = cstage + lane * 128;
@@ -336,13 +440,13 @@ __global__ void __launch_bounds__(kTileThreads, 1)
     }
 }
 
-template <int BN, bool GROUPED, int STAGES, int NBUF>
+template <int BN, int GMODE, int STAGES, int NBUF>
 static dg_status_t launch_tile_impl(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream) {
-    using L = TileSmem<BN, STAGES, NBUF>;
+    using L = TileSmem<BN, STAGES, NBUF, GMODE>;
     static_assert(L::kDynamicBytes <= 232448, "shared memory budget");
     static_assert(STAGES % 2 == 0 && NBUF % 2 == 0, "each MMA thread must own its stages and buffers");
     CUtensorMap tmA, tmB, tmC;
-    const uint64_t b_rows = GROUPED ? static_cast<uint64_t>(a.G) * a.N : static_cast<uint64_t>(a.N);
+    const uint64_t b_rows = GMODE != kDense ? static_cast<uint64_t>(a.G) * a.N : static_cast<uint64_t>(a.N);
     dg_status_t st;
     st = make_tmap_2d(&tmA, a.A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.M, a.K, 128, 128,
                       CU_TENSOR_MAP_SWIZZLE_128B);
@@ -359,6 +463,10 @@ static dg_status_t launch_tile_impl(const GemmArgs &a, const DeviceInfo &dev, cu
     p.sA = a.sA;
     p.sB = a.sB;
     p.offsets = a.offsets;
+    p.masked_m = a.masked_m;
+    p.m_max = static_cast<int>(a.m_max);
+    p.mb_max = static_cast<int>((a.m_max + 127) / 128);
+    p.C = static_cast<__nv_bfloat16 *>(a.C);
     p.G = a.G;
     p.num_m_cap = static_cast<int>((a.M + 127) / 128);
     p.num_n_tiles = static_cast<int>((a.N + BN - 1) / BN);
@@ -370,7 +478,7 @@ static dg_status_t launch_tile_impl(const GemmArgs &a, const DeviceInfo &dev, cu
     p.status = ctl.status;
     p.debug_flags = ctl.debug_flags;
 
-    auto kernel = tile_gemm_kernel<BN, GROUPED, STAGES, NBUF>;
+    auto kernel = tile_gemm_kernel<BN, GMODE, STAGES, NBUF>;
     static thread_local int configured_device = -1;
     int device = 0;
     cudaGetDevice(&device);
@@ -384,19 +492,24 @@ static dg_status_t launch_tile_impl(const GemmArgs &a, const DeviceInfo &dev, cu
         if (128 * regs_producer<BN>() + 256 * regs_epilogue<BN>() > kTileThreads * fa.numRegs) return DG_ERR_CUDA;
         configured_device = device;
     }
-    const int64_t tiles = static_cast<int64_t>(p.num_m_cap) * p.num_n_tiles;
+    // kMasked: the counts live on the device, so size the grid for full slabs
+    const int64_t m_blocks = GMODE == kMasked ? static_cast<int64_t>(a.G) * p.mb_max : p.num_m_cap;
+    const int64_t tiles = m_blocks * p.num_n_tiles;
     const int grid = static_cast<int>(tiles < dev.num_sms ? tiles : dev.num_sms);
     kernel<<<grid, kTileThreads, L::kDynamicBytes, stream>>>(tmA, tmB, tmC, p);
     return cudaGetLastError() == cudaSuccess ? DG_OK : DG_ERR_CUDA;
 }
 
-dg_status_t launch_tile_gemm(const GemmArgs &a, bool grouped, const DeviceInfo &dev, cudaStream_t stream) {
+dg_status_t launch_tile_gemm(const GemmArgs &a, int group, const DeviceInfo &dev, cudaStream_t stream) {
     // BN = 256 columns per tile unless the matrix is narrower (fewer idle columns).
     const bool narrow = a.N <= 128;
-    if (grouped) {
-        return narrow ? launch_tile_impl<128, true, 6, 4>(a, dev, stream) : launch_tile_impl<256, true, 4, 2>(a, dev, stream);
-    }
-    return narrow ? launch_tile_impl<128, false, 6, 4>(a, dev, stream) : launch_tile_impl<256, false, 4, 2>(a, dev, stream);
+    if (group == kContiguous)
+        return narrow ? launch_tile_impl<128, kContiguous, 6, 4>(a, dev, stream)
+                      : launch_tile_impl<256, kContiguous, 4, 2>(a, dev, stream);
+    if (group == kMasked)
+        return narrow ? launch_tile_impl<128, kMasked, 6, 4>(a, dev, stream)
+                      : launch_tile_impl<256, kMasked, 4, 2>(a, dev, stream);
+    return narrow ? launch_tile_impl<128, kDense, 6, 4>(a, dev, stream) : launch_tile_impl<256, kDense, 4, 2>(a, dev, stream);
 }
 
 }  // namespace dg

@@ -145,6 +145,29 @@ dg_status_t dg_fp8_grouped_gemm_contiguous(const uint8_t *A, const float *sA,
                                            int64_t N, int64_t K, cudaStream_t stream);
 
 /*
+ * MoE masked grouped block-scaled GEMM (2kiu.com/news/5461879 §2.2: the experts
+ * share N and K, only M varies, and from call to call): expert g owns a slab of
+ * M_max rows of A and C and uses its first masked_m[g] rows, a count read on the
+ * device (so an earlier kernel on `stream` may write it, with no host sync).
+ * For those rows
+ *   C[g][m][n] = bf16( sum_kb sA[g][m/128][kb] * sB[g][n/128][kb] *
+ *                      sum_k A[g][m][k] * B[g][n][k] ).
+ * Only m-blocks holding tokens are computed; rows at or past masked_m[g] of C
+ * are not written, and rows past masked_m[g] of A may hold anything.
+ *
+ * A  : [G][M_max][K] E4M3, 16-byte aligned.  sA : [G][ceil(M_max/128)][ceil(K/128)] FP32.
+ * B  : [G][N][K] E4M3.                       sB : [G][N/128][ceil(K/128)] FP32.
+ * C  : [G][M_max][N] BF16 out.
+ * masked_m : DEVICE int32 [G]; counts outside [0, M_max] are clamped to it.
+ * 1 <= G <= 256, M_max >= 0, N % 128 == 0, K % 16 == 0, K > 0.
+ * M_max == 0 or N == 0 is a no-op.
+ */
+dg_status_t dg_fp8_grouped_gemm_masked(const uint8_t *A, const float *sA,
+                                       const uint8_t *B, const float *sB,
+                                       void *C_bf16, const int32_t *masked_m, int G,
+                                       int64_t M_max, int64_t N, int64_t K, cudaStream_t stream);
+
+/*
  * Kernel selection for the dense GEMM, for tests and measurement.  AUTO is the
  * dispatch dg_fp8_gemm_blockscaled uses: SKINNY for M <= 128, else PAIR.
  *   TILE    persistent single-CTA kernel, 128 x 256 (128 x 128 if N <= 128) tiles;

@@ -68,5 +68,12 @@ def test_host_validation_without_device(lib):
     assert lib.dg_fp8_gemm_blockscaled_bf16a(null, null, null, null, null, null, 8, 24, 128, null) == 2
     assert lib.dg_fp8_gemm_blockscaled_bf16a(null, null, null, null, null, null, 0, 16, 128, null) == 0
     assert lib.dg_fp8_gemm_blockscaled_bf16a(null, null, null, null, null, null, 8, 16, 128, null) == 1
+    # masked MoE: G in [1, 256], N % 128, K % 16, then pointers
+    assert lib.dg_fp8_grouped_gemm_masked(null, null, null, null, null, null, 0, 128, 128, 128, null) == 2
+    assert lib.dg_fp8_grouped_gemm_masked(null, null, null, null, null, null, 257, 128, 128, 128, null) == 2
+    assert lib.dg_fp8_grouped_gemm_masked(null, null, null, null, null, null, 2, 128, 64, 128, null) == 2
+    assert lib.dg_fp8_grouped_gemm_masked(null, null, null, null, null, null, 2, 128, 128, 40, null) == 2
+    assert lib.dg_fp8_grouped_gemm_masked(null, null, null, null, null, null, 2, 0, 128, 128, null) == 0
+    assert lib.dg_fp8_grouped_gemm_masked(null, null, null, null, null, null, 2, 128, 128, 128, null) == 1
     odd = ctypes.c_void_p(0x1001)
     assert lib.dg_fp8_gemm_blockscaled(odd, odd, odd, odd, odd, 8, 16, 128, null) == 3

@@ -1,0 +1,110 @@
+"""GPU parity of the masked MoE GEMM (per-expert token counts read on the device)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fp8_block_scaled_scales_b200 import binding, inputs
+
+from parity import c_f64, check, dev, oracle_quant
+
+pytestmark = pytest.mark.gpu
+
+
+def quantized(w, junk_seed=None):
+    qa, sa = oracle_quant(w.A)   # per expert slab: [G][M_max][K], [G][ceil(M_max/128)][Kb]
+    qb, sb = oracle_quant(w.B)
+    if junk_seed is not None:
+        # rows past each count may hold anything, NaN codes included: no output may see them
+        rng = np.random.default_rng(junk_seed)
+        for g in range(w.G):
+            c = int(w.counts[g])
+            qa[g, c:] = rng.integers(0, 256, size=qa[g, c:].shape, dtype=np.uint8)
+    return qa, sa, qb, sb
+
+
+def run(qa, sa, qb, sb, counts, fill=-3.0):
+    G, Mmax, K = qa.shape
+    N = qb.shape[1]
+    C = torch.full((G, Mmax, N), fill, dtype=torch.bfloat16, device="cuda")
+    mm = torch.from_numpy(np.asarray(counts, dtype=np.int32)).cuda()
+    binding.grouped_gemm_masked(dev(qa), dev(sa), dev(qb), dev(sb), mm, C=C)
+    torch.cuda.synchronize()
+    assert binding.last_device_status() == 0
+    return C
+
+
+@pytest.mark.parametrize("G,Mmax,N,K,counts", [
+    (4, 200, 256, 256, [0, 200, 77, 129]),
+    (4, 256, 128, 4000, [256, 0, 1, 128]),      # narrow N (128-column tiles), K tail
+    (3, 130, 384, 640, [130, 2, 65]),
+    (1, 1000, 512, 384, [999]),
+])
+def test_masked_small_full_compare(G, Mmax, N, K, counts):
+    w = inputs.masked_custom(G, Mmax, N, K, counts, seed=9500 + G + Mmax + N)
+    qa, sa, qb, sb = quantized(w, junk_seed=9600 + G)
+    C = c_f64(run(qa, sa, qb, sb, counts))
+    ref = oracle.masked_gemm_ref(qa, sa, qb, sb, counts)
+    real = np.concatenate([ref[g, :counts[g]] for g in range(G)])
+    got = np.concatenate([C[g, :counts[g]] for g in range(G)])
+    rms = float(np.sqrt(np.mean(real ** 2)))
+    check(got, real, rms, "masked real rows")
+    for g in range(G):
+        assert np.all(C[g, counts[g]:] == -3.0), f"expert {g}: rows past its count were written"
+
+
+def test_masked_counts_clamped_and_written_on_device():
+    """Counts come from an earlier kernel on the stream; out-of-range ones are clamped."""
+    G, Mmax, N, K = 3, 256, 256, 256
+    counts = [300, -4, 100]  # clamped to 256, 0, 100
+    w = inputs.masked_custom(G, Mmax, N, K, [256, 0, 100], seed=9700)
+    qa, sa, qb, sb = quantized(w)
+    mm = torch.tensor([0, 0, 0], dtype=torch.int32, device="cuda")
+    mm += torch.tensor(counts, dtype=torch.int32, device="cuda")  # stream-ordered device write
+    C = torch.full((G, Mmax, N), -3.0, dtype=torch.bfloat16, device="cuda")
+    binding.grouped_gemm_masked(dev(qa), dev(sa), dev(qb), dev(sb), mm, C=C)
+    torch.cuda.synchronize()
+    assert binding.last_device_status() == 0
+    ref = oracle.masked_gemm_ref(qa, sa, qb, sb, np.array(counts))
+    c = c_f64(C)
+    check(c[0], ref[0], None, "expert 0 (count clamped to M_max)")
+    assert np.all(c[1] == -3.0)
+    check(c[2, :100], ref[2, :100], None, "expert 2")
+    assert np.all(c[2, 100:] == -3.0)
+
+
+def test_masked_equals_contiguous_kernel_bitwise():
+    """Same tokens in the contiguous layout: the same tile arithmetic, so the same bits."""
+    G, Mmax, N, K = 3, 384, 512, 512
+    counts = np.array([384, 130, 7])
+    w = inputs.masked_custom(G, Mmax, N, K, counts, seed=9800)
+    qa, sa, qb, sb = quantized(w)
+    Cm = run(qa, sa, qb, sb, counts)
+    padded = (counts + 127) // 128 * 128
+    off = np.concatenate([[0], np.cumsum(padded)]).astype(np.int32)
+    Ac = np.zeros((int(off[-1]), K), np.uint8)
+    sAc = np.ones((int(off[-1]) // 128, K // 128), np.float32)
+    for g in range(G):
+        Ac[off[g]:off[g] + counts[g]] = qa[g, :counts[g]]
+        sAc[off[g] // 128:off[g] // 128 + padded[g] // 128] = sa[g, :padded[g] // 128]
+    Cc = binding.grouped_gemm_contiguous(dev(Ac), dev(sAc), dev(qb), dev(sb), dev(off))
+    torch.cuda.synchronize()
+    for g in range(G):
+        a = Cm[g, :counts[g]].view(torch.int16)
+        b = Cc[off[g]:off[g] + counts[g]].view(torch.int16)
+        assert torch.equal(a, b), f"expert {g}"
+
+
+def test_moe_masked_g8_workload_sampled():
+    w = inputs.moe_masked_g8()
+    qa, sa, qb, sb = quantized(w, junk_seed=9900)
+    C = c_f64(run(qa, sa, qb, sb, w.counts))
+    rng = np.random.default_rng(0)
+    for g in range(w.G):
+        c = int(w.counts[g])
+        if c == 0:
+            continue
+        rows = np.unique(np.concatenate([[0, c - 1], rng.integers(0, c, 6)])).astype(np.int64)
+        ref = oracle.gemm_ref(qa[g], sa[g], qb[g], sb[g], rows=rows)
+        check(C[g][rows], ref, None, f"moe_masked_g8 expert {g}")
+        assert np.all(C[g, c:] == -3.0)
