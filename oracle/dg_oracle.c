@@ -147,14 +147,33 @@ void dgo_bf16_from_double_array(const double *x, int64_t n, uint16_t *out)
 /* ------------------------------------------------------------------------- */
 /* Block quantizer: BF16 [R][C] -> E4M3 codes [R][C] + FP32 scales [Rb][Cb]   */
 /* ------------------------------------------------------------------------- */
+/*
+ * Blocks of brows x blk elements: brows = blk is the 128x128 form; brows = 1 gives
+ * one scale per row and 128-column group ("per-group, 128 elements a group",
+ * demingchina.com/news/60142 §5.2), S [R][Cb].
+ */
+static void quantize_blocks(const uint16_t *X, int64_t R, int64_t C, int64_t brows, int64_t blk,
+                            uint8_t *Q, float *S);
+
 void dgo_quantize_blockwise(const uint16_t *X, int64_t R, int64_t C, int64_t blk,
                             uint8_t *Q, float *S)
 {
+    quantize_blocks(X, R, C, blk, blk, Q, S);
+}
+
+void dgo_quantize_groups(const uint16_t *X, int64_t R, int64_t C, int64_t blk, uint8_t *Q, float *S)
+{
+    quantize_blocks(X, R, C, 1, blk, Q, S);
+}
+
+static void quantize_blocks(const uint16_t *X, int64_t R, int64_t C, int64_t brows, int64_t blk,
+                            uint8_t *Q, float *S)
+{
     init_mag();
-    int64_t Rb = (R + blk - 1) / blk, Cb = (C + blk - 1) / blk;
+    int64_t Rb = (R + brows - 1) / brows, Cb = (C + blk - 1) / blk;
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t br = 0; br < Rb; ++br) {
-        int64_t r0 = br * blk, r1 = r0 + blk < R ? r0 + blk : R;
+        int64_t r0 = br * brows, r1 = r0 + brows < R ? r0 + brows : R;
         for (int64_t bc = 0; bc < Cb; ++bc) {
             int64_t c0 = bc * blk, c1 = c0 + blk < C ? c0 + blk : C;
             float amax = 0.0f;
@@ -203,10 +222,36 @@ static void decode_rows(const uint8_t *X, int64_t K, int64_t row, double *out, c
     for (int64_t k = 0; k < K; ++k) out[k] = tab[X[row * K + k]];
 }
 
+/*
+ * The same formula with A's scales per `ablk` rows: sA[m / ablk][kb].  ablk = blk
+ * is the 128x128 form above; ablk = 1 gives one scale per row and 128-wide K group
+ * ("per-group, 128 elements a group", demingchina.com/news/60142 §5.2), sA [M][Kb].
+ */
+static void gemm_ref_impl(const uint8_t *A, const float *sA, int64_t ablk, const uint8_t *B, const float *sB,
+                          int64_t M, int64_t N, int64_t K, int64_t blk,
+                          const int64_t *rows, int64_t nrows, const int64_t *cols, int64_t ncols,
+                          double *out);
+
 void dgo_gemm_ref(const uint8_t *A, const float *sA, const uint8_t *B, const float *sB,
                   int64_t M, int64_t N, int64_t K, int64_t blk,
                   const int64_t *rows, int64_t nrows, const int64_t *cols, int64_t ncols,
                   double *out)
+{
+    gemm_ref_impl(A, sA, blk, B, sB, M, N, K, blk, rows, nrows, cols, ncols, out);
+}
+
+void dgo_gemm_ref_rowscale(const uint8_t *A, const float *sA, const uint8_t *B, const float *sB,
+                           int64_t M, int64_t N, int64_t K, int64_t blk,
+                           const int64_t *rows, int64_t nrows, const int64_t *cols, int64_t ncols,
+                           double *out)
+{
+    gemm_ref_impl(A, sA, 1, B, sB, M, N, K, blk, rows, nrows, cols, ncols, out);
+}
+
+static void gemm_ref_impl(const uint8_t *A, const float *sA, int64_t ablk, const uint8_t *B, const float *sB,
+                          int64_t M, int64_t N, int64_t K, int64_t blk,
+                          const int64_t *rows, int64_t nrows, const int64_t *cols, int64_t ncols,
+                          double *out)
 {
     double tab[256];
     dgo_e4m3_table(tab);
@@ -234,7 +279,7 @@ void dgo_gemm_ref(const uint8_t *A, const float *sA, const uint8_t *B, const flo
                     double p = 0.0;
                     int64_t k1 = (kb + 1) * blk < K ? (kb + 1) * blk : K;
                     for (int64_t k = kb * blk; k < k1; ++k) p += Ad[k] * b[k];
-                    double s = (double)sA[(m / blk) * Kb + kb] * (double)sB[(n / blk) * Kb + kb];
+                    double s = (double)sA[(m / ablk) * Kb + kb] * (double)sB[(n / blk) * Kb + kb];
                     ref += s * p;
                 }
                 out[i * ncols + j] = ref;

@@ -13,6 +13,11 @@ Functions and the passages they follow:
   gemm_ref            block formula with per-K-block promotion, 2kiu.com/news/5461879
                       §2.1 and §3.3 (FP32 accumulate, segmented accumulation);
                       demingchina.com/news/60142 §3.1 (scales multiplied back at output)
+  quantize_groups     one scale per row and 128-element group ("per-group, 128 elements a
+                      group", demingchina.com/news/60142 §5.2); otherwise as above
+  gemm_ref_rowscale   gemm_ref with those per-row A scales (B keeps 128x128 blocks)
+  masked_gemm_ref     masked MoE layout: expert g's first masked_m[g] rows, the dense
+                      formula per expert (2kiu.com/news/5461879 §2.2)
   grouped_gemm_ref    experts stored contiguously by expert id, one long matrix
                       (nxmr.cn/news/132300 §2.2), N and K fixed, M varies
                       (2kiu.com/news/5461879 §2.2)
@@ -52,7 +57,9 @@ def _load():
     lib.dgo_bf16_from_double.argtypes = [ctypes.c_double]
     lib.dgo_bf16_from_double_array.argtypes = [vp, i64, vp]
     lib.dgo_quantize_blockwise.argtypes = [vp, i64, i64, i64, vp, vp]
+    lib.dgo_quantize_groups.argtypes = [vp, i64, i64, i64, vp, vp]
     lib.dgo_gemm_ref.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, vp, i64, vp, i64, vp]
+    lib.dgo_gemm_ref_rowscale.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, vp, i64, vp, i64, vp]
     lib.dgo_grouped_gemm_ref.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp, i64, vp, i64, vp]
     lib.dgo_init()
     _lib = lib
@@ -121,6 +128,19 @@ def quantize_blockwise(x_bf16_bits: np.ndarray):
     return q, s
 
 
+def quantize_groups(x_bf16_bits: np.ndarray):
+    """BF16 [R][C] -> (E4M3 codes [R][C], FP32 scales [R][Cb]): one scale per row and
+    128-column group, s = fl32(amax/448) over the group's elements."""
+    lib = _load()
+    x = np.ascontiguousarray(x_bf16_bits, dtype=np.uint16)
+    assert x.ndim == 2
+    R, C = x.shape
+    q = np.empty((R, C), dtype=np.uint8)
+    s = np.empty((R, -(-C // BLK)), dtype=np.float32)
+    lib.dgo_quantize_groups(_ptr(x), R, C, BLK, _ptr(q), _ptr(s))
+    return q, s
+
+
 # --------------------------------------------------------------------------- GEMM
 def _idx(a, n):
     if a is None:
@@ -150,6 +170,26 @@ def gemm_ref(A, sA, B, sB, rows=None, cols=None) -> np.ndarray:
     lib.dgo_gemm_ref(_ptr(A), _ptr(sA), _ptr(B), _ptr(sB), M, N, K, BLK,
                      None if r is None else _ptr(r), nr, None if c is None else _ptr(c), nc,
                      _ptr(out))
+    return out
+
+
+def gemm_ref_rowscale(A, sA, B, sB, rows=None, cols=None) -> np.ndarray:
+    """gemm_ref with one A scale per row and K block: sA [M][ceil(K/128)]."""
+    lib = _load()
+    A = np.ascontiguousarray(A, dtype=np.uint8)
+    B = np.ascontiguousarray(B, dtype=np.uint8)
+    sA = np.ascontiguousarray(sA, dtype=np.float32)
+    sB = np.ascontiguousarray(sB, dtype=np.float32)
+    M, K = A.shape
+    N, K2 = B.shape
+    assert K == K2 and K > 0
+    assert sA.shape == (M, -(-K // BLK)) and sB.shape == (-(-N // BLK), -(-K // BLK))
+    r, nr = _idx(rows, M)
+    c, nc = _idx(cols, N)
+    out = np.empty((nr, nc), dtype=np.float64)
+    lib.dgo_gemm_ref_rowscale(_ptr(A), _ptr(sA), _ptr(B), _ptr(sB), M, N, K, BLK,
+                              None if r is None else _ptr(r), nr, None if c is None else _ptr(c), nc,
+                              _ptr(out))
     return out
 
 

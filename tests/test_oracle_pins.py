@@ -50,8 +50,9 @@ def random_scales(rng, shape):
     return (rng.uniform(0.5, 2.0, size=shape) * 2.0 ** rng.integers(-12, 2, size=shape)).astype(np.float32)
 
 
-def exact_ref(A, sA, B, sB, with_abs=False):
+def exact_ref(A, sA, B, sB, with_abs=False, a_rows=128):
     """Exact block formula as Fractions: integer K-block partials, Fraction scale sum.
+    A's scale of row m is sA[m // a_rows] (128: 128x128 blocks, 1: one per row).
 
     With with_abs, also returns sum_kb |s_kb * P_kb| (float), the scale of the FP64
     summation error bound."""
@@ -71,7 +72,7 @@ def exact_ref(A, sA, B, sB, with_abs=False):
         for n in range(N):
             acc = Fraction(0)
             for kb in range(Kb):
-                t = fa[m // 128][kb] * fb[n // 128][kb] * int(parts[kb][m, n])
+                t = fa[m // a_rows][kb] * fb[n // 128][kb] * int(parts[kb][m, n])
                 acc += t
                 absum[m, n] += abs(float(t)) / 2.0 ** 18
             out[m][n] = acc / (1 << 18)
@@ -468,3 +469,61 @@ def test_masked_ref_equals_contiguous_ref_on_packed_rows():
     # clamping: a count past M_max acts as M_max, a negative one as 0
     clamped = oracle.masked_gemm_ref(A, sA, B, sB, np.array([-5, 999, 77, 129]))
     assert np.array_equal(clamped[1], got[1]) and np.all(np.isnan(clamped[0]))
+
+
+# ------------------------------------------------ per-row (1 x 128 group) A scales
+@pytest.mark.parametrize("R,C", [(1, 16), (130, 384), (64, 1040)])
+def test_group_quantizer_matches_torch_division_and_cast(R, C):
+    """One scale per row and 128-column group: torch's FP32 amax / 448 and its FP32
+    division + float8 cast (a library routine) give the same scales and codes."""
+    x = _quant_case(R, C, 7000 + R + C, outlier=True)
+    x[0, :16] = 0.0  # a partial group of zeros when C == 16
+    q, s = oracle.quantize_groups(_bits(x))
+    xf = x.to(torch.float32)
+    Cb = -(-C // 128)
+    xp = torch.zeros((R, Cb * 128))
+    xp[:, :C] = xf
+    g = xp.reshape(R, Cb, 128)
+    amax = g.abs().amax(dim=2)
+    scale = torch.where(amax == 0, torch.ones_like(amax), amax / torch.tensor(448.0))
+    assert np.array_equal(s, scale.numpy())
+    want = (g / scale[:, :, None]).reshape(R, Cb * 128)[:, :C].to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(q, want)
+    # every non-zero group holds a code at +-448
+    for r in range(R):
+        for b in range(Cb):
+            if amax[r, b] > 0:
+                assert np.any((q[r, 128 * b:128 * b + 128] & 0x7F) == 0x7E)
+
+
+@pytest.mark.parametrize("M,N,K,seed", [(7, 5, 256, 41), (130, 129, 272, 42), (33, 300, 128, 43)])
+def test_rowscale_gemm_against_exact_brute_force(M, N, K, seed):
+    rng = np.random.default_rng(seed)
+    Kb = -(-K // 128)
+    A = random_finite_codes(rng, (M, K))
+    B = random_finite_codes(rng, (N, K))
+    sA = random_scales(rng, (M, Kb))
+    sB = random_scales(rng, (-(-N // 128), Kb))
+    ref = oracle.gemm_ref_rowscale(A, sA, B, sB)
+    exact, absum = exact_ref(A, sA, B, sB, with_abs=True, a_rows=1)
+    ex = np.array([[float(v) for v in row] for row in exact])
+    assert np.all(np.abs(ref - ex) <= 2 * (Kb + 1) * 2.0 ** -53 * absum)
+
+
+def test_rowscale_gemm_equals_block_gemm_when_rows_share_scales():
+    """Per-row scales that repeat the 128-row block's scale give the block form, bit for bit."""
+    rng = np.random.default_rng(44)
+    M, N, K = 300, 200, 384
+    A = random_finite_codes(rng, (M, K))
+    B = random_finite_codes(rng, (N, K))
+    sA = random_scales(rng, (3, 3))
+    sB = random_scales(rng, (2, 3))
+    rows_scales = np.ascontiguousarray(sA[np.arange(M) // 128])
+    assert np.array_equal(oracle.gemm_ref_rowscale(A, rows_scales, B, sB), oracle.gemm_ref(A, sA, B, sB))
+    # and a row's own scale acts on that row alone
+    sr = rows_scales.copy()
+    sr[5] *= 4
+    a = oracle.gemm_ref_rowscale(A, sr, B, sB)
+    b = oracle.gemm_ref_rowscale(A, rows_scales, B, sB)
+    assert np.array_equal(np.delete(a, 5, 0), np.delete(b, 5, 0))
+    assert np.allclose(a[5], 4 * b[5], rtol=1e-15, atol=0)
