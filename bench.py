@@ -74,11 +74,14 @@ def load_peaks():
 
 # ------------------------------------------------------------------ workloads
 WORKLOADS = ("dense_4096_outliers", "dense_512", "dense_8192", "skinny_m1", "skinny_m16", "skinny_m64",
-             "skinny_m128", "moe_g8", "moe_g64_zipf", "moe_masked_g8")
+             "skinny_m128", "moe_g8", "moe_g64_zipf", "moe_masked_g8",
+             "dense_4096_outliers_1x128")
 
 
 def make_workload(name):
     from fp8_block_scaled_scales_b200 import inputs
+    if name.endswith("_1x128"):  # the same data, per-token activation scales
+        name = name[:-len("_1x128")]
     if name == "dense_4096_outliers":
         return inputs.dense_4096_outliers()
     if name == "dense_512":
@@ -184,7 +187,7 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- CPU oracle
-def oracle_sample(w, rows_sample: int, seed: int = 0):
+def oracle_sample(w, rows_sample: int, seed: int = 0, rowscale: bool = False):
     """Time the CPU oracle on `rows_sample` rows of the workload (quantize those rows
     of A, then the block-scaled GEMM of those rows against all of B).  Returns
     (seconds, flops done, threads, description).  B's quantization is not timed
@@ -230,8 +233,12 @@ def oracle_sample(w, rows_sample: int, seed: int = 0):
     rows = min(rows_sample, w.M)
     rows = max(rows, 1)
     t0 = time.perf_counter()
-    qa, sa = oracle.quantize_blockwise(inputs.bf16_bits(w.A[:rows]))
-    ref = oracle.gemm_ref(qa, sa, qb, sb)
+    if rowscale:
+        qa, sa = oracle.quantize_groups(inputs.bf16_bits(w.A[:rows]))
+        ref = oracle.gemm_ref_rowscale(qa, sa, qb, sb)
+    else:
+        qa, sa = oracle.quantize_blockwise(inputs.bf16_bits(w.A[:rows]))
+        ref = oracle.gemm_ref(qa, sa, qb, sb)
     out = oracle.bf16_from_double(ref)
     dt = time.perf_counter() - t0
     del out
@@ -289,7 +296,10 @@ def run_dg(args):
     flops, gemm_bytes, rows_a, cfg = workload_facts(w)
     grouped = isinstance(w, Grouped)
     masked = isinstance(w, Masked)
-    skinny = not (grouped or masked) and w.M <= 128
+    rowscale = args.workload.endswith("_1x128")  # one A scale per row and 128-K group
+    if rowscale:
+        cfg = dict(cfg, workload=args.workload, a_scales="one per row and 128-K group (K-block-major)")
+    skinny = not (grouped or masked or rowscale) and w.M <= 128
     fused = skinny and w.M <= FUSED_MAX_M  # one launch: the GEMM quantizes A itself
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream()
@@ -308,6 +318,8 @@ def run_dg(args):
         mm = torch.from_numpy(w.counts.astype(np.int32)).to(dev)
     qa = torch.empty((rows_a, w.K), dtype=torch.uint8, device=dev)
     sa = torch.empty((-(-rows_a // 128), -(-w.K // 128)), dtype=torch.float32, device=dev)
+    if rowscale:
+        sa = torch.empty((-(-w.K // 128), rows_a), dtype=torch.float32, device=dev)  # K-block-major
     C = torch.empty((rows_a, w.N), dtype=torch.bfloat16, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
 
@@ -317,14 +329,22 @@ def run_dg(args):
                                         C=C.view(w.G, w.M_max, w.N))
         elif grouped:
             binding.grouped_gemm_contiguous(qa, sa, qb, sb, off, C=C)
+        elif rowscale:
+            binding.gemm_1x128(qa, sa, qb, sb, C=C)
         else:
             binding.gemm_blockscaled(qa, sa, qb, sb, C=C)
+
+    def quantize_a(x):
+        if rowscale:
+            binding.quantize_1x128(x, q=qa, s_t=sa)
+        else:
+            binding.quantize_blockwise(x, q=qa, s=sa)
 
     def step(x):
         if fused:
             binding.gemm_blockscaled_bf16a(x, qb, sb, C=C, QA=qa, sA=sa)
         else:
-            binding.quantize_blockwise(x, q=qa, s=sa)
+            quantize_a(x)
             gemm()
 
     for _ in range(args.warmup):
@@ -355,7 +375,7 @@ def run_dg(args):
             if fused:
                 step(A)  # the fused kernel is the whole step
             else:
-                binding.quantize_blockwise(A, q=qa, s=sa)
+                quantize_a(A)
                 ev[i][1].record(stream)
                 gemm()
             ev[i][2].record(stream)
@@ -440,7 +460,7 @@ def run_dg(args):
     if cs is not None:
         out["clocks"] = cs
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        dt, fl, cores, desc = oracle_sample(w, args.oracle_rows or default_oracle_rows(w))
+        dt, fl, cores, desc = oracle_sample(w, args.oracle_rows or default_oracle_rows(w), rowscale=rowscale)
         if unit == "GB/s":
             v = (gemm_bytes * fl / flops) / dt / 1e9
         else:
@@ -465,7 +485,7 @@ def run_reference(args):
     rows = args.oracle_rows or max(1, default_oracle_rows(w) // 4)
     times = []
     for i in range(args.warmup + args.steps):
-        dt, fl, cores, desc = oracle_sample(w, rows, seed=i)
+        dt, fl, cores, desc = oracle_sample(w, rows, seed=i, rowscale=args.workload.endswith("_1x128"))
         if i >= args.warmup:
             times.append((dt, fl))
     dt = sum(t for t, _ in times)

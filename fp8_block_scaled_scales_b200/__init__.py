@@ -4,6 +4,6 @@ The compute lives in libdg.so (hand-written CUDA kernels behind a C ABI,
 include/dg.h); this package is its Python binding plus the seeded input
 generators used by the tests and the benchmark.
 """
-from .binding import (DGError, gemm_blockscaled, gemm_blockscaled_bf16a,  # noqa: F401
+from .binding import (DGError, gemm_1x128, gemm_blockscaled, gemm_blockscaled_bf16a,  # noqa: F401
                       grouped_gemm_contiguous, grouped_gemm_masked, last_device_status, quantize_blockwise,
-                      set_kernel_control, version)
+                      quantize_1x128, set_kernel_control, version)

@@ -23,7 +23,8 @@ KERNELS = {"auto": 0, "tile": 1, "skinny": 2, "pair": 3}
 
 # every symbol include/dg.h declares
 EXPORTS = ("dg_quantize_blockwise", "dg_fp8_gemm_blockscaled", "dg_fp8_gemm_blockscaled_bf16a",
-           "dg_fp8_grouped_gemm_contiguous", "dg_fp8_grouped_gemm_masked",
+           "dg_fp8_grouped_gemm_contiguous", "dg_fp8_grouped_gemm_masked", "dg_quantize_1x128",
+           "dg_fp8_gemm_1x128", "dg_fp8_gemm_1x128_select",
            "dg_fp8_gemm_blockscaled_select", "dg_status_string", "dg_get_last_device_status",
            "dg_version", "dg_test_set_kernel_control")
 
@@ -53,9 +54,13 @@ def lib() -> ctypes.CDLL:
     L.dg_fp8_gemm_blockscaled_bf16a.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp]
     L.dg_fp8_grouped_gemm_contiguous.argtypes = [vp, vp, vp, vp, vp, vp, i64, i32, i64, i64, vp]
     L.dg_fp8_grouped_gemm_masked.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, i64, i64, vp]
+    L.dg_quantize_1x128.argtypes = [vp, i64, i64, vp, vp, vp]
+    L.dg_fp8_gemm_1x128.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp]
+    L.dg_fp8_gemm_1x128_select.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, vp]
     for f in ("dg_quantize_blockwise", "dg_fp8_gemm_blockscaled", "dg_fp8_gemm_blockscaled_select",
               "dg_fp8_gemm_blockscaled_bf16a",
-              "dg_fp8_grouped_gemm_contiguous", "dg_fp8_grouped_gemm_masked", "dg_get_last_device_status"):
+              "dg_fp8_grouped_gemm_contiguous", "dg_fp8_grouped_gemm_masked", "dg_get_last_device_status",
+              "dg_quantize_1x128", "dg_fp8_gemm_1x128", "dg_fp8_gemm_1x128_select"):
         getattr(L, f).restype = ctypes.c_int
     L.dg_get_last_device_status.argtypes = [vp]
     L.dg_status_string.restype = ctypes.c_char_p
@@ -151,6 +156,31 @@ def grouped_gemm_contiguous(A, sA, B, sB, offsets, C=None, stream=None):
     _check(lib().dg_fp8_grouped_gemm_contiguous(_p(A), _p(sA), _p(B), _p(sB), _p(C), _p(offsets), Mcap, G,
                                                 N, K, _stream(stream)),
            "dg_fp8_grouped_gemm_contiguous")
+    return C
+
+
+def quantize_1x128(x: torch.Tensor, q: torch.Tensor | None = None, s_t: torch.Tensor | None = None,
+                   stream=None):
+    """BF16 [R][C] -> (E4M3 codes [R][C], FP32 scales [ceil(C/128)][R]), one per row and group."""
+    R, C = x.shape
+    if q is None:
+        q = torch.empty((R, C), dtype=torch.uint8, device=x.device)
+    if s_t is None:
+        s_t = torch.empty(((C + 127) // 128, R), dtype=torch.float32, device=x.device)
+    _check(lib().dg_quantize_1x128(_p(x), R, C, _p(_u8(q)), _p(s_t), _stream(stream)), "dg_quantize_1x128")
+    return q, s_t
+
+
+def gemm_1x128(A, sA_t, B, sB, C=None, kernel: str = "auto", stream=None):
+    """C[M][N] (bf16) from A with per-token scales sA_t [ceil(K/128)][M] and 128x128 B scales."""
+    A, B = _u8(A), _u8(B)
+    M, K = A.shape
+    N = B.shape[0]
+    if C is None:
+        C = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    _check(lib().dg_fp8_gemm_1x128_select(_p(A), _p(sA_t), _p(B), _p(sB), _p(C), M, N, K, KERNELS[kernel],
+                                          _stream(stream)),
+           "dg_fp8_gemm_1x128")
     return C
 
 

@@ -147,6 +147,18 @@ dg_status_t dg_quantize_blockwise(const void *X_bf16, int64_t rows, int64_t cols
     return launch_quantize(X_bf16, rows, cols, Q, S, dev, stream);
 }
 
+dg_status_t dg_quantize_1x128(const void *X_bf16, int64_t rows, int64_t cols, uint8_t *Q, float *S_t,
+                              cudaStream_t stream) {
+    if (rows < 0 || cols < 0 || cols % 16 != 0) return DG_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return DG_OK;
+    if (!X_bf16 || !Q || !S_t) return DG_ERR_INVALID_ARG;
+    if (!aligned(X_bf16, 16) || !aligned(Q, 16) || !aligned(S_t, 4)) return DG_ERR_ALIGNMENT;
+    DeviceInfo dev;
+    dg_status_t st = current_device(&dev, nullptr);
+    if (st != DG_OK) return st;
+    return launch_quantize_groups(X_bf16, rows, cols, Q, S_t, dev, stream);
+}
+
 static dg_status_t check_gemm_common(const uint8_t *A, const float *sA, const uint8_t *B, const float *sB,
                                      const void *C) {
     if (!A || !sA || !B || !sB || !C) return DG_ERR_INVALID_ARG;
@@ -181,6 +193,30 @@ dg_status_t dg_fp8_gemm_blockscaled_select(const uint8_t *A, const float *sA, co
 dg_status_t dg_fp8_gemm_blockscaled(const uint8_t *A, const float *sA, const uint8_t *B, const float *sB,
                                     void *C_bf16, int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
     return dg_fp8_gemm_blockscaled_select(A, sA, B, sB, C_bf16, M, N, K, DG_KERNEL_AUTO, stream);
+}
+
+dg_status_t dg_fp8_gemm_1x128_select(const uint8_t *A, const float *sA_t, const uint8_t *B, const float *sB,
+                                     void *C_bf16, int64_t M, int64_t N, int64_t K, dg_kernel_t kernel,
+                                     cudaStream_t stream) {
+    if (M < 0 || N < 0 || K <= 0 || K % 16 != 0 || N % 16 != 0) return DG_ERR_SHAPE;
+    if (M > 0x7FFFFFFFLL || N > 0x7FFFFFFFLL || K > 0x7FFFFFFFLL) return DG_ERR_SHAPE;
+    if (kernel != DG_KERNEL_AUTO && kernel != DG_KERNEL_TILE && kernel != DG_KERNEL_PAIR) return DG_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) return DG_OK;
+    dg_status_t st = check_gemm_common(A, sA_t, B, sB, C_bf16);
+    if (st != DG_OK) return st;
+    DeviceInfo dev;
+    st = current_device(&dev, nullptr);
+    if (st != DG_OK) return st;
+    GemmArgs a = {A, sA_t, B, sB, C_bf16, nullptr, M, N, K, 0};
+    a.row_scales = true;
+    if (kernel == DG_KERNEL_AUTO) kernel = M <= 128 ? DG_KERNEL_TILE : DG_KERNEL_PAIR;
+    if (kernel == DG_KERNEL_TILE) return launch_tile_gemm(a, 0, dev, stream);
+    return N <= 128 ? launch_pair_gemm_n128(a, dev, stream) : launch_pair_gemm(a, dev, stream);
+}
+
+dg_status_t dg_fp8_gemm_1x128(const uint8_t *A, const float *sA_t, const uint8_t *B, const float *sB, void *C_bf16,
+                              int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
+    return dg_fp8_gemm_1x128_select(A, sA_t, B, sB, C_bf16, M, N, K, DG_KERNEL_AUTO, stream);
 }
 
 dg_status_t dg_fp8_gemm_blockscaled_bf16a(const void *A_bf16, const uint8_t *B, const float *sB, void *C_bf16,

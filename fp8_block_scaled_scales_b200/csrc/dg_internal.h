@@ -48,6 +48,7 @@ struct GemmArgs {
     int G;                   // grouped only
     const int32_t *masked_m = nullptr;  // masked only: tokens per expert (device)
     int64_t m_max = 0;                  // masked only: rows per expert slab
+    bool row_scales = false;            // dense only: sA is [ceil(K/128)][M], one scale per row
 };
 
 // group: 0 dense, 1 grouped-contiguous, 2 masked
@@ -61,6 +62,9 @@ dg_status_t launch_skinny_gemm(const GemmArgs &a, const DeviceInfo &dev, cudaStr
 constexpr int64_t kFusedMaxM = 32;
 dg_status_t launch_skinny_gemm_fused(const GemmArgs &a, const void *A_bf16, uint8_t *qa_out, float *sa_out,
                                      const DeviceInfo &dev, cudaStream_t stream);
+// one scale per row and 128-column group, written K-block-major: St[ceil(cols/128)][rows]
+dg_status_t launch_quantize_groups(const void *X, int64_t rows, int64_t cols, uint8_t *Q, float *St,
+                                   const DeviceInfo &dev, cudaStream_t stream);
 dg_status_t launch_quantize(const void *X, int64_t rows, int64_t cols, uint8_t *Q, float *S,
                             const DeviceInfo &dev, cudaStream_t stream);
 

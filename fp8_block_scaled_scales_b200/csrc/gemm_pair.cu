@@ -87,7 +87,9 @@ __device__ __forceinline__ void settle_after_abort() {
     }
 }
 
-template <int BN, int STAGES, int NBUF>
+// ROWS: sA holds one scale per row of A and K block, K-block-major (sA[kb][m]);
+// each epilogue thread promotes its row with its own scale.
+template <int BN, int STAGES, int NBUF, bool ROWS>
 __global__ void __launch_bounds__(kPairThreads, 1)
     pair_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, const PairParams p) {
@@ -228,14 +230,23 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             const int nb128 = col0 / 128;
             const bool valid = nb128 < p.Nb && mb < p.num_m;
             ScaleStream scales;
-            scales.start(p.sA + static_cast<int64_t>(valid ? mb : 0) * Kb,
+            scales.start(ROWS ? nullptr : p.sA + static_cast<int64_t>(valid ? mb : 0) * Kb,
                          p.sB + static_cast<int64_t>(valid ? nb128 : 0) * Kb, 0, valid ? Kb : 0);
+            // ROWS: this thread's row scale, loaded one K block ahead
+            const int my_row = mb * 128 + quarter * 32 + lane;
+            const bool row_ok = ROWS && valid && my_row < p.M;
+            float sa_next = row_ok ? __ldg(p.sA + my_row) : 0.0f;
 #pragma unroll
             for (int i = 0; i < kColsPerWarp / 2; ++i) acc[i] = make_float2(0.0f, 0.0f);
             for (int kb = 0; kb < Kb; ++kb, ++kc) {
                 const int buf = kc % NBUF;
                 const uint32_t v = static_cast<uint32_t>(kc / NBUF);
-                const float scale = scales.scale(kb, kb);
+                float scale = scales.scale(kb, kb);
+                if (ROWS) {
+                    const float sa = sa_next;
+                    sa_next = (row_ok && kb + 1 < Kb) ? __ldg(p.sA + static_cast<int64_t>(kb + 1) * p.M + my_row) : 0.0f;
+                    scale = sa * scale;  // fl32(sA[row][kb] * sB[n/128][kb])
+                }
                 const float2 s2 = make_float2(scale, scale);
                 if (!mbar_wait(&tfull[buf], v & 1u, abort_flag, p.timeout_ns)) {
                     record_failure(p.status, kStatusTimeout, 24 + static_cast<int>(rank), kc);
@@ -310,7 +321,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     }
 }
 
-template <int BN, int STAGES, int NBUF>
+template <int BN, int STAGES, int NBUF, bool ROWS>
 static dg_status_t launch_pair_impl(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream) {
     using L = PairSmem<BN, STAGES, NBUF>;
     static_assert(L::kDynamicBytes <= 232448, "shared memory budget");
@@ -339,7 +350,7 @@ static dg_status_t launch_pair_impl(const GemmArgs &a, const DeviceInfo &dev, cu
     p.status = ctl.status;
     p.debug_flags = ctl.debug_flags;
 
-    auto kernel = pair_gemm_kernel<BN, STAGES, NBUF>;
+    auto kernel = pair_gemm_kernel<BN, STAGES, NBUF, ROWS>;
     static thread_local int configured_device = -1;
     static thread_local int max_pairs = 0;
     int device = 0;
@@ -377,11 +388,13 @@ static dg_status_t launch_pair_impl(const GemmArgs &a, const DeviceInfo &dev, cu
 }
 
 dg_status_t launch_pair_gemm(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream) {
-    return launch_pair_impl<256, 6, 2>(a, dev, stream);
+    return a.row_scales ? launch_pair_impl<256, 6, 2, true>(a, dev, stream)
+                        : launch_pair_impl<256, 6, 2, false>(a, dev, stream);
 }
 
 dg_status_t launch_pair_gemm_n128(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream) {
-    return launch_pair_impl<128, 8, 4>(a, dev, stream);
+    return a.row_scales ? launch_pair_impl<128, 8, 4, true>(a, dev, stream)
+                        : launch_pair_impl<128, 8, 4, false>(a, dev, stream);
 }
 
 }  // namespace dg

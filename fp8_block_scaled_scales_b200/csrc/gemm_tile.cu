@@ -167,7 +167,9 @@ __device__ __forceinline__ TileInfo resolve_tile(const TileParams &p, const int 
     return ti;
 }
 
-template <int BN, int GMODE, int STAGES, int NBUF>
+// ROWS (dense only): sA holds one scale per row of A and K block, K-block-major
+// (sA[kb][m]); each epilogue thread promotes its row with its own scale.
+template <int BN, int GMODE, int STAGES, int NBUF, bool ROWS>
 __global__ void __launch_bounds__(kTileThreads, 1)
     tile_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, const TileParams p) {
@@ -343,14 +345,23 @@ __global__ void __launch_bounds__(kTileThreads, 1)
             const bool n_valid = nb128 < p.Nb;
             const int sb_row = ti.sb_row + nb128;
             ScaleStream scales;
-            scales.start(p.sA + static_cast<int64_t>(ti.sa_row) * Kb, p.sB + static_cast<int64_t>(sb_row) * Kb, 0,
-                         n_valid ? Kb : 0);
+            scales.start(ROWS ? nullptr : p.sA + static_cast<int64_t>(ti.sa_row) * Kb,
+                         p.sB + static_cast<int64_t>(sb_row) * Kb, 0, n_valid ? Kb : 0);
+            // ROWS: this thread's row scale, loaded one K block ahead
+            const int my_row = ti.a_row + quarter * 32 + lane;
+            const bool row_ok = ROWS && my_row < p.M;
+            float sa_next = row_ok ? __ldg(p.sA + my_row) : 0.0f;
 #pragma unroll
             for (int i = 0; i < kColsPerWarp / 2; ++i) acc[i] = make_float2(0.0f, 0.0f);
             for (int kb = 0; kb < Kb; ++kb, ++kc) {
                 const int buf = kc % NBUF;
                 const uint32_t v = static_cast<uint32_t>(kc / NBUF);
-                const float scale = scales.scale(kb, kb);
+                float scale = scales.scale(kb, kb);
+                if (ROWS) {
+                    const float sa = sa_next;
+                    sa_next = (row_ok && kb + 1 < Kb) ? __ldg(p.sA + static_cast<int64_t>(kb + 1) * p.M + my_row) : 0.0f;
+                    scale = sa * scale;  // fl32(sA[row][kb] * sB[n/128][kb])
+                }
                 const float2 s2 = make_float2(scale, scale);
                 if (!mbar_wait(&tfull[buf], v & 1u, abort_flag, p.timeout_ns)) {
                     record_failure(p.status, kStatusTimeout, 2, kc);
@@ -440,7 +451,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
     }
 }
 
-template <int BN, int GMODE, int STAGES, int NBUF>
+template <int BN, int GMODE, int STAGES, int NBUF, bool ROWS = false>
 static dg_status_t launch_tile_impl(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream) {
     using L = TileSmem<BN, STAGES, NBUF, GMODE>;
     static_assert(L::kDynamicBytes <= 232448, "shared memory budget");
@@ -478,7 +489,7 @@ static dg_status_t launch_tile_impl(const GemmArgs &a, const DeviceInfo &dev, cu
     p.status = ctl.status;
     p.debug_flags = ctl.debug_flags;
 
-    auto kernel = tile_gemm_kernel<BN, GMODE, STAGES, NBUF>;
+    auto kernel = tile_gemm_kernel<BN, GMODE, STAGES, NBUF, ROWS>;
     static thread_local int configured_device = -1;
     int device = 0;
     cudaGetDevice(&device);
@@ -509,6 +520,9 @@ dg_status_t launch_tile_gemm(const GemmArgs &a, int group, const DeviceInfo &dev
     if (group == kMasked)
         return narrow ? launch_tile_impl<128, kMasked, 6, 4>(a, dev, stream)
                       : launch_tile_impl<256, kMasked, 4, 2>(a, dev, stream);
+    if (a.row_scales)
+        return narrow ? launch_tile_impl<128, kDense, 6, 4, true>(a, dev, stream)
+                      : launch_tile_impl<256, kDense, 4, 2, true>(a, dev, stream);
     return narrow ? launch_tile_impl<128, kDense, 6, 4>(a, dev, stream) : launch_tile_impl<256, kDense, 4, 2>(a, dev, stream);
 }
 

@@ -70,6 +70,43 @@ __global__ void __launch_bounds__(kQuantThreads)
     }
 }
 
+// One scale per row and 128-column group ("per-group, 128 elements a group",
+// demingchina.com/news/60142 §5.2): the same conversion with the group as the
+// block.  Sixteen lanes own a group (16 bytes = 8 BF16 each; a row's group is 256
+// contiguous bytes), so the amax needs only shuffles.  Groups run row by row, the
+// groups of a row side by side; the scales go out K-block-major, St[kb][row], the
+// layout in which the GEMM's epilogue reads one per row with coalesced loads.
+__global__ void __launch_bounds__(kQuantThreads)
+    quantize_groups_kernel(const uint16_t *__restrict__ X, int64_t R, int64_t C, int64_t Cb, int64_t groups,
+                           uint8_t *__restrict__ Q, float *__restrict__ St) {
+    const int tid = static_cast<int>(threadIdx.x);
+    const int64_t gi = static_cast<int64_t>(blockIdx.x) * (kQuantThreads / 16) + (tid >> 4);
+    const bool group_ok = gi < groups;
+    const int64_t row = group_ok ? gi / Cb : 0;
+    const int64_t kb = group_ok ? gi - row * Cb : 0;
+    const int64_t col = kb * 128 + (tid & 15) * 8;
+    const bool present = group_ok && col < C;  // C % 16 == 0: an 8-column piece is whole or absent
+    const uint4 v = present ? __ldg(reinterpret_cast<const uint4 *>(X + row * C + col)) : make_uint4(0, 0, 0, 0);
+    uint32_t amax_bits = amax_bits_of(amax_fold8(0u, v));
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) amax_bits = max(amax_bits, __shfl_xor_sync(0xFFFFFFFFu, amax_bits, o));
+    const BlockScale bs = block_scale(amax_bits);
+    if (present) *reinterpret_cast<uint2 *>(Q + row * C + col) = quantize8(v, bs);
+    if (group_ok && (tid & 15) == 0) St[kb * R + row] = bs.s;
+}
+
+dg_status_t launch_quantize_groups(const void *X, int64_t rows, int64_t cols, uint8_t *Q, float *St,
+                                   const DeviceInfo &dev, cudaStream_t stream) {
+    (void)dev;
+    const int64_t Cb = (cols + 127) / 128;
+    const int64_t groups = rows * Cb;
+    const int64_t blocks = (groups + kQuantThreads / 16 - 1) / (kQuantThreads / 16);
+    if (blocks > 0x7FFFFFFFLL) return DG_ERR_SHAPE;
+    quantize_groups_kernel<<<static_cast<unsigned>(blocks), kQuantThreads, 0, stream>>>(
+        static_cast<const uint16_t *>(X), rows, cols, Cb, groups, Q, St);
+    return cudaGetLastError() == cudaSuccess ? DG_OK : DG_ERR_CUDA;
+}
+
 dg_status_t launch_quantize(const void *X, int64_t rows, int64_t cols, uint8_t *Q, float *S,
                             const DeviceInfo &dev, cudaStream_t stream) {
     (void)dev;

@@ -145,6 +145,35 @@ dg_status_t dg_fp8_grouped_gemm_contiguous(const uint8_t *A, const float *sA,
                                            int64_t N, int64_t K, cudaStream_t stream);
 
 /*
+ * Per-token activation quantizer: one FP32 scale per row and 128-column group
+ * ("per-group, 128 elements a group", demingchina.com/news/60142 §5.2), with the
+ * same arithmetic as dg_quantize_blockwise on that 1 x 128 block:
+ *   s = fl32(amax / 448) (1 if amax == 0);  q = E4M3_rn_satfinite(fl32(x / s)).
+ *
+ * X_bf16 : [rows][cols] BF16, 16-byte aligned.
+ * Q      : [rows][cols] E4M3 out, 16-byte aligned.
+ * S_t    : [ceil(cols/128)][rows] FP32 out, K-block-major (the transpose of the
+ *          natural [rows][groups]): the layout dg_fp8_gemm_1x128 reads.
+ * rows >= 0, cols >= 0, cols % 16 == 0; an empty matrix is a no-op.
+ */
+dg_status_t dg_quantize_1x128(const void *X_bf16, int64_t rows, int64_t cols,
+                              uint8_t *Q, float *S_t, cudaStream_t stream);
+
+/*
+ * Block-scaled GEMM with per-token A scales (demingchina.com/news/60142 §5.2)
+ * and 128x128 B scales:
+ *   C[m][n] = bf16( sum_kb sA_t[kb][m] * sB[n/128][kb] *
+ *                   sum_{k in block kb} A[m][k] * B[n][k] )
+ *
+ * A    : [M][K] E4M3.            sA_t : [ceil(K/128)][M] FP32 (from dg_quantize_1x128).
+ * B, sB, C and the shape rules as in dg_fp8_gemm_blockscaled.
+ * M <= 128 runs the tile kernel, larger M the CTA-pair kernel.
+ */
+dg_status_t dg_fp8_gemm_1x128(const uint8_t *A, const float *sA_t,
+                              const uint8_t *B, const float *sB, void *C_bf16,
+                              int64_t M, int64_t N, int64_t K, cudaStream_t stream);
+
+/*
  * MoE masked grouped block-scaled GEMM (2kiu.com/news/5461879 §2.2: the experts
  * share N and K, only M varies, and from call to call): expert g owns a slab of
  * M_max rows of A and C and uses its first masked_m[g] rows, a count read on the
@@ -180,6 +209,13 @@ dg_status_t dg_fp8_gemm_blockscaled_select(const uint8_t *A, const float *sA,
                                            const uint8_t *B, const float *sB, void *C_bf16,
                                            int64_t M, int64_t N, int64_t K,
                                            dg_kernel_t kernel, cudaStream_t stream);
+
+/* dg_fp8_gemm_1x128 with the kernel chosen: AUTO, TILE or PAIR (SKINNY gives
+ * DG_ERR_INVALID_ARG), for tests and measurement. */
+dg_status_t dg_fp8_gemm_1x128_select(const uint8_t *A, const float *sA_t,
+                                     const uint8_t *B, const float *sB, void *C_bf16,
+                                     int64_t M, int64_t N, int64_t K, dg_kernel_t kernel,
+                                     cudaStream_t stream);
 
 /* Human-readable name of a status code (static storage). */
 const char *dg_status_string(dg_status_t status);

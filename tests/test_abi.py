@@ -75,5 +75,11 @@ def test_host_validation_without_device(lib):
     assert lib.dg_fp8_grouped_gemm_masked(null, null, null, null, null, null, 2, 128, 128, 40, null) == 2
     assert lib.dg_fp8_grouped_gemm_masked(null, null, null, null, null, null, 2, 0, 128, 128, null) == 0
     assert lib.dg_fp8_grouped_gemm_masked(null, null, null, null, null, null, 2, 128, 128, 128, null) == 1
+    # per-token scales
+    assert lib.dg_quantize_1x128(null, 4, 17, null, null, null) == 2
+    assert lib.dg_quantize_1x128(null, 0, 16, null, null, null) == 0
+    assert lib.dg_fp8_gemm_1x128(null, null, null, null, null, 8, 16, 100, null) == 2
+    assert lib.dg_fp8_gemm_1x128(null, null, null, null, null, 8, 16, 128, null) == 1
+    assert lib.dg_fp8_gemm_1x128_select(null, null, null, null, null, 8, 16, 128, 2, null) == 1
     odd = ctypes.c_void_p(0x1001)
     assert lib.dg_fp8_gemm_blockscaled(odd, odd, odd, odd, odd, 8, 16, 128, null) == 3
