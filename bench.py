@@ -46,10 +46,10 @@ FP8_OVER_BF16 = 2.0  # nominal dense FP8 / BF16 tensor throughput ratio on B200
 # (profiles/), keyed by workload and the hash of that kernel's source file; a
 # kernel changed since the capture reports null.
 NCU_TRAFFIC = {
-    # pair_gemm_kernel<256,6,2>, dense 4096^3: 33.594880 MB read + 2.309376 MB written
-    ("dense_4096_outliers", "gemm_pair.cu", "50658734f922265e"): 35904256,
-    # skinny_gemm_kernel<16,8,8>, M=16 N=K=4096: 16.872704 MB read, 0 written (C stays in L2)
-    ("skinny_m16", "gemm_skinny.cu", "5d0f81b2578f1a2c"): 16872704,
+    # pair_gemm_kernel<256,6,2,0>, dense 4096^3: 33.590272 MB read + 3.567872 MB written
+    ("dense_4096_outliers", "gemm_pair.cu", "4c0b5c0743766ffc"): 37158144,
+    # skinny_gemm_kernel<16,8,8,1> (A quantized inside), M=16 N=K=4096: 16.953600 MB read, 0 written
+    ("skinny_m16", "gemm_skinny.cu", "3903e55d474f370d"): 16953600,
 }
 
 
