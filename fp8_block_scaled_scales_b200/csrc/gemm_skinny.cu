@@ -41,6 +41,7 @@ struct SkinnyParams {
     int splits;
     uint64_t timeout_ns;
     int *status;  // device status word
+    int debug_flags;  // bit 0 (tests): the producer never fills stage 0, so a wait must time out
     // FUSED only: BF16 A [M][K], and the codes / scales written by the first N block
     const uint16_t *Xa;
     int K;
@@ -196,6 +197,7 @@ __global__ void __launch_bounds__(skinny_threads<FUSED>(), 1)
                 *abort_flag = 1;
                 break;
             }
+            if ((p.debug_flags & 1) && i == 0) continue;  // test hook: stage 0 never filled
             mbar_arrive_expect_tx(&full[s], FUSED ? L::kWBytes : L::kWBytes + L::kXBytes);
             tma_load_2d(smem + L::kOffW + s * L::kWBytes, &tmW, &full[s], kb * 128, nb * 128);
             if (!FUSED) tma_load_2d(smem + L::kOffX + s * L::kXBytes, &tmX, &full[s], kb * 128, 0);
@@ -501,6 +503,7 @@ static dg_status_t launch_skinny_impl(const GemmArgs &a, const uint16_t *Xa, uin
     p.splits = S;
     p.timeout_ns = kernel_control().timeout_ns;
     p.status = kernel_control().status;
+    p.debug_flags = kernel_control().debug_flags;
     p.Xa = Xa;
     p.K = static_cast<int>(a.K);
     p.qa_out = qa_out;
