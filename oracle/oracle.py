@@ -1,4 +1,4 @@
-"""Python driver of the CPU oracle for the FP8 (E4M3) 128x128 block-scaled GEMM.
+"""Python wrapper of the CPU oracle for the FP8 (E4M3) 128x128 block-scaled GEMM.
 
 TEST INFRASTRUCTURE ONLY: only the test suite, the smoke check and the benchmark's
 CPU-baseline leg may import this module.  It shares no code with the CUDA library
