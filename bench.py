@@ -39,7 +39,7 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-FUSED_MAX_M = 32  # the library quantizes A inside the skinny GEMM up to this M
+FUSED_MAX_M = 1  # the library quantizes A inside the skinny GEMM up to this M
 E2E_PIPELINE_MIN_BYTES = 4 << 20  # host<->device bytes per step above which e2e overlaps copies
 L2_FLUSH_BYTES = 256 << 20
 FP8_OVER_BF16 = 2.0  # nominal dense FP8 / BF16 tensor throughput ratio on B200
@@ -50,8 +50,10 @@ FP8_OVER_BF16 = 2.0  # nominal dense FP8 / BF16 tensor throughput ratio on B200
 NCU_TRAFFIC = {
     # pair_gemm_kernel<256,6,2,0>, dense 4096^3: 33.590272 MB read + 3.567872 MB written
     ("dense_4096_outliers", "gemm_pair.cu", "4c0b5c0743766ffc"): 37158144,
-    # skinny_gemm_kernel<16,8,8,1> (A quantized inside), M=16 N=K=4096: 16.954112 MB read, 0 written
-    ("skinny_m16", "gemm_skinny.cu", "2f320dc51362dd29"): 16954112,
+    # skinny_gemm_kernel<16,8,8,1> (A quantized inside), M=1 N=K=4096: 16.831232 MB read, 0 written
+    ("skinny_m1", "gemm_skinny.cu", "7a4728a38640b1ea"): 16831232,
+    # skinny_gemm_kernel<16,8,8,0>, M=16 N=K=4096: 16.873216 MB read, 0 written
+    ("skinny_m16", "gemm_skinny.cu", "7a4728a38640b1ea"): 16873216,
     # tile_gemm_kernel<256,kMasked,4,2,0>, moe_masked_g8: 211.488512 MB read + 112.432384 MB written
     ("moe_masked_g8", "gemm_tile.cu", "64df6b0f04c7b8da"): 323920896,
 }

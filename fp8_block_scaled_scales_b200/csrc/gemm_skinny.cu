@@ -535,8 +535,8 @@ dg_status_t launch_skinny_gemm(const GemmArgs &a, const DeviceInfo &dev, cudaStr
 dg_status_t launch_skinny_gemm_fused(const GemmArgs &a, const void *A_bf16, uint8_t *qa_out, float *sa_out,
                                      const DeviceInfo &dev, cudaStream_t stream) {
     const uint16_t *x = static_cast<const uint16_t *>(A_bf16);
-    if (a.M <= 16) return launch_skinny_impl<16, 8, 8, true>(a, x, qa_out, sa_out, dev, stream);
-    if (a.M <= kFusedMaxM) return launch_skinny_impl<32, 8, 8, true>(a, x, qa_out, sa_out, dev, stream);
+    static_assert(kFusedMaxM <= 16, "one token slab of 16 rows");
+    if (a.M <= kFusedMaxM) return launch_skinny_impl<16, 8, 8, true>(a, x, qa_out, sa_out, dev, stream);
     return DG_ERR_SHAPE;
 }
 

@@ -111,9 +111,10 @@ dg_status_t dg_fp8_gemm_blockscaled(const uint8_t *A, const float *sA,
  *          Caller-owned: they receive A's codes and scales (the library allocates
  *          nothing).
  * Shapes as in dg_fp8_gemm_blockscaled (N % 16 == 0, K % 16 == 0, K > 0).
- * M <= 32: one launch -- the skinny kernel quantizes A inside its producer
+ * M == 1: one launch -- the skinny kernel quantizes A inside its producer
  * stage (no separate pass over A).  Larger M: the block quantizer, then the
- * FP8 GEMM, on `stream`.  M == 0 or N == 0 is a no-op.
+ * FP8 GEMM, on `stream` (faster from M = 2 on, measured).  M == 0 or N == 0 is
+ * a no-op.
  */
 dg_status_t dg_fp8_gemm_blockscaled_bf16a(const void *A_bf16, const uint8_t *B, const float *sB,
                                           void *C_bf16, uint8_t *QA, float *sA,

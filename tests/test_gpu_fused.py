@@ -1,6 +1,6 @@
 """GPU parity of the GEMM that takes BF16 activations and quantizes them itself.
 
-For M <= 32 one kernel quantizes A inside its producer stage; it must give the
+For M = 1 one kernel quantizes A inside its producer stage; it must give the
 block quantizer's codes and scales bit for bit, and the same C, bit for bit, as
 the FP8 GEMM run on those codes (same kernel family, same promotion order), and
 C within tolerance of the oracle.  Larger M runs the quantizer, then the tile GEMM.
