@@ -27,6 +27,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -49,19 +50,34 @@ FP8_OVER_BF16 = 2.0  # nominal dense FP8 / BF16 tensor throughput ratio on B200
 # kernel changed since the capture reports null.
 NCU_TRAFFIC = {
     # pair_gemm_kernel<256,6,2,0>, dense 4096^3: 33.590272 MB read + 3.567872 MB written
-    ("dense_4096_outliers", "gemm_pair.cu", "4c0b5c0743766ffc"): 37158144,
+    ("dense_4096_outliers", "gemm_pair.cu", "50ae5d72260e6871"): 37158144,
     # skinny_gemm_kernel<16,8,8,1> (A quantized inside), M=1 N=K=4096: 16.831232 MB read, 0 written
-    ("skinny_m1", "gemm_skinny.cu", "7a4728a38640b1ea"): 16831232,
+    ("skinny_m1", "gemm_skinny.cu", "6dff96e6ca9b1718"): 16831232,
     # skinny_gemm_kernel<16,8,8,0>, M=16 N=K=4096: 16.873216 MB read, 0 written
-    ("skinny_m16", "gemm_skinny.cu", "7a4728a38640b1ea"): 16873216,
+    ("skinny_m16", "gemm_skinny.cu", "6dff96e6ca9b1718"): 16873216,
     # tile_gemm_kernel<256,kMasked,4,2,0>, moe_masked_g8: 211.488512 MB read + 112.432384 MB written
-    ("moe_masked_g8", "gemm_tile.cu", "64df6b0f04c7b8da"): 323920896,
+    ("moe_masked_g8", "gemm_tile.cu", "33f6a825e56547a0"): 323920896,
 }
 
 
+KERNEL_HEADERS = ("dg_device.cuh", "quant_e4m3.cuh")  # device code the kernels include
+
+
+def _code_only(text: str) -> str:
+    """Source without comments and blank lines: a comment edit leaves the kernel as it was."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def kernel_source_hash(fname: str) -> str:
-    with open(os.path.join(ROOT, "fp8_block_scaled_scales_b200", "csrc", fname), "rb") as fh:
-        return hashlib.sha256(fh.read()).hexdigest()[:16]
+    """Hash of a kernel's code (its .cu file and the shared device headers), which keys
+    the DRAM traffic measured by ncu: once the code changes, the figure is dropped."""
+    h = hashlib.sha256()
+    for f in (fname,) + KERNEL_HEADERS:
+        with open(os.path.join(ROOT, "fp8_block_scaled_scales_b200", "csrc", f)) as fh:
+            h.update(_code_only(fh.read()).encode())
+    return h.hexdigest()[:16]
 
 
 def ncu_traffic(workload: str, kernel_file: str):

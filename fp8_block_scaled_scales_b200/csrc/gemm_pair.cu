@@ -1,4 +1,5 @@
-// CTA-pair (cta_group::2) FP8 block-scaled GEMM tile kernel for sm_100a, dense form.
+// CTA-pair (cta_group::2) FP8 block-scaled GEMM tile kernel for sm_100a, dense form,
+// with 128x128 A scales or (ROWS) one A scale per row and K block.
 //
 // Same method and roles as the single-CTA tile kernel (gemm_tile.cu): per 128-wide
 // K block the tensor cores produce P_kb in FP32 in tensor memory and the epilogue
@@ -25,8 +26,10 @@
 //   tfull[b]   in both CTAs: the MMA commit (multicast) arrives on both.
 // Two threads of the even CTA issue the MMAs, alternating K blocks.
 //   tempty[b]  even CTA only: all 16 epilogue warps of the pair arrive on it.
-// All waits are CTA-scope polls of the waiting CTA's own barrier; the peer's
-// remote arrivals carry cluster-scope release semantics.
+// All waits are CTA-scope polls of the waiting CTA's own barrier.  The remote
+// arrivals only hand back tensor memory, whose reads are ordered by tcgen05
+// fences, not generic memory, so they use the default CTA-scope semantics (a
+// cluster-scope release fenced every arrival and halved the throughput).
 #include <cuda_bf16.h>
 
 #include "dg_device.cuh"

@@ -1,5 +1,6 @@
 // Persistent, warp-specialised FP8 (E4M3) block-scaled GEMM tile kernel for
-// sm_100a, dense and MoE grouped-contiguous forms.
+// sm_100a: dense, MoE grouped-contiguous and MoE masked forms, with 128x128 A
+// scales or (ROWS, dense) one A scale per row and K block.
 //
 // Method (2kiu.com/news/5461879 §2.1, §3.3; demingchina.com/news/60142 §3.1):
 //   C[m][n] = bf16( sum_kb sA[m/128][kb] * sB[n/128][kb] * P_kb[m][n] ),
@@ -19,11 +20,13 @@
 //   warps 1-2   MMA issuers: one thread each, alternating K blocks; per K block
 //               four tcgen05.mma (K = 32 each) into that K block's TMEM partial
 //               buffer, then one commit to the buffer's "full" barrier.
-//   warp 3      idle.
+//   warp 3      (kMasked) builds the m-block prefix table, then idles.
 //   warps 4-11  epilogue: per kb, free the shared-memory stage, tcgen05.ld the
 //               partial 16 columns at a time (software-pipelined against the FMAs),
 //               release the TMEM buffer as soon as the last load has landed, and
-//               acc += s * P_kb with packed FP32 FMAs; after the last kb, round to
+//               acc += s * P_kb with packed FP32 FMAs (ROWS: s is the thread's
+//               row scale, loaded two K blocks ahead, times the B scale); after
+//               the last kb, round to
 //               BF16, stage in swizzled shared memory and TMA-store.  Warp w reads
 //               TMEM lanes 32*(w%4).. (the lane quarter its warp id allows) and
 //               columns half (w-4)/4 of the tile.
