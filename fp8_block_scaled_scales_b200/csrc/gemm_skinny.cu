@@ -25,6 +25,9 @@
 // thus needs no launch of its own (2kiu.com/news/5461879 §5: activation scales
 // are recomputed on every call).  The CTAs of the first N block also write the
 // codes and scales out, so the caller gets the same Q, S as from the quantizer.
+// Every N block's CTAs repeat the quantization of their K range, and each K
+// block's conversion sits on its MMA's critical path, so the one launch pays
+// only for a single token row; the library uses it for M = 1.
 #include <cuda_bf16.h>
 
 #include "dg_device.cuh"
