@@ -179,3 +179,28 @@ def test_skinny_workload(M):
 @pytest.mark.slow
 def test_dense_8192_workload():
     _sampled_rows_check(inputs.dense_8192(), n_random=24)
+
+
+@pytest.mark.parametrize("M,N,K,kernel", [(512, 768, 1024, "pair"), (512, 768, 1024, "tile"),
+                                          (64, 1024, 2048, "skinny")])
+def test_per_tensor_special_case_matches_cublaslt(M, N, K, kernel):
+    """All A scales equal and all B scales equal: the method is then per-tensor-scaled FP8
+    GEMM, which cuBLASLt computes (torch._scaled_mm, a library routine).  A cross-check of
+    the whole harness: our kernel, cuBLASLt and the oracle must agree within tolerance."""
+    d = inputs.dense_custom(M, N, K, seed=8600 + M + N + K)
+    qa, _ = oracle_quant(d.A)
+    qb, _ = oracle_quant(d.B)
+    a_s, b_s = np.float32(0.0137), np.float32(0.00211)
+    sa = np.full((-(-M // 128), K // 128), a_s, np.float32)
+    sb = np.full((-(-N // 128), K // 128), b_s, np.float32)
+    c = c_f64(run(qa, sa, qb, sb, kernel=kernel))
+    A8 = dev(qa).view(torch.float8_e4m3fn)
+    B8 = dev(qb).view(torch.float8_e4m3fn)
+    c_lt = torch._scaled_mm(A8, B8.t(), scale_a=torch.tensor(float(a_s), device="cuda"),
+                            scale_b=torch.tensor(float(b_s), device="cuda"), out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    ref = oracle.gemm_ref(qa, sa, qb, sb)
+    check(c, ref, None, f"{kernel} per-tensor vs oracle")
+    check(c_f64(c_lt), ref, None, "cuBLASLt per-tensor vs oracle")
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    check(c, c_f64(c_lt), rms, f"{kernel} vs cuBLASLt")
