@@ -16,7 +16,7 @@ from parity import c_f64, check, dev, oracle_quant
 
 pytestmark = pytest.mark.gpu
 
-SHAPES = [(1, 4096, 4096), (16, 4096, 4096), (17, 512, 640), (64, 1040, 768), (100, 256, 256),
+SHAPES = [(1, 4096, 4096), (1, 272, 144), (1, 4096, 4000), (16, 4096, 4096), (17, 512, 640), (64, 1040, 768), (100, 256, 256),
           (128, 4096, 512), (33, 128, 4096), (5, 272, 144), (48, 384, 4000), (300, 512, 1152)]
 
 

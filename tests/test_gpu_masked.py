@@ -108,3 +108,19 @@ def test_moe_masked_g8_workload_sampled():
         ref = oracle.gemm_ref(qa[g], sa[g], qb[g], sb[g], rows=rows)
         check(C[g][rows], ref, None, f"moe_masked_g8 expert {g}")
         assert np.all(C[g, c:] == -3.0)
+
+
+def test_masked_largest_expert_count():
+    """G = 256, the most the prefix table holds: many empty and one-token experts."""
+    G, Mmax, N, K = 256, 128, 128, 128
+    rng = np.random.default_rng(9950)
+    counts = rng.choice([0, 0, 1, 7, 128, 64], size=G)
+    w = inputs.masked_custom(G, Mmax, N, K, counts, seed=9951)
+    qa, sa, qb, sb = quantized(w, junk_seed=9952)
+    C = c_f64(run(qa, sa, qb, sb, counts))
+    ref = oracle.masked_gemm_ref(qa, sa, qb, sb, counts)
+    real = np.concatenate([ref[g, :counts[g]] for g in range(G) if counts[g]])
+    got = np.concatenate([C[g, :counts[g]] for g in range(G) if counts[g]])
+    check(got, real, float(np.sqrt(np.mean(real ** 2))), "masked G=256")
+    for g in range(G):
+        assert np.all(C[g, counts[g]:] == -3.0)
