@@ -83,3 +83,24 @@ def test_host_validation_without_device(lib):
     assert lib.dg_fp8_gemm_1x128_select(null, null, null, null, null, 8, 16, 128, 2, null) == 1
     odd = ctypes.c_void_p(0x1001)
     assert lib.dg_fp8_gemm_blockscaled(odd, odd, odd, odd, odd, 8, 16, 128, null) == 3
+
+
+def declared_signatures():
+    """{name: number of parameters} for every function include/dg.h declares."""
+    text = open(os.path.join(ROOT, "include", "dg.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(dg_\w+)\s*\(([^()]*)\)\s*;", text):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else len(params.split(","))
+    return out
+
+
+def test_binding_argument_lists_match_the_header(lib):
+    """A parameter added on one side only would shift every argument after it."""
+    sigs = declared_signatures()
+    assert set(sigs) == set(binding.EXPORTS)
+    for name, n in sigs.items():
+        argtypes = getattr(lib, name).argtypes
+        if argtypes is not None:
+            assert len(argtypes) == n, (name, len(argtypes), n)
