@@ -104,3 +104,26 @@ def test_binding_argument_lists_match_the_header(lib):
         argtypes = getattr(lib, name).argtypes
         if argtypes is not None:
             assert len(argtypes) == n, (name, len(argtypes), n)
+
+
+def _ctype_of(param: str):
+    p = param.strip()
+    if "*" in p or p.startswith("cudaStream_t"):
+        return ctypes.c_void_p
+    base = p.rsplit(" ", 1)[0].replace("const ", "").strip()
+    return {"int64_t": ctypes.c_int64, "uint64_t": ctypes.c_uint64, "int": ctypes.c_int,
+            "dg_kernel_t": ctypes.c_int, "dg_status_t": ctypes.c_int}[base]
+
+
+def test_binding_argument_types_match_the_header(lib):
+    """Pointer, 32- and 64-bit integer parameters must be passed as such: an int64_t
+    bound as c_int leaves the upper half of the register undefined."""
+    text = open(os.path.join(ROOT, "include", "dg.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    for m in re.finditer(r"\b(dg_\w+)\s*\(([^()]*)\)\s*;", text):
+        params = m.group(2).strip()
+        if params in ("", "void"):
+            continue
+        want = [_ctype_of(x) for x in params.split(",")]
+        got = list(getattr(lib, m.group(1)).argtypes)
+        assert got == want, (m.group(1), got, want)
