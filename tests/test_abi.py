@@ -83,6 +83,18 @@ def test_host_validation_without_device(lib):
     assert lib.dg_fp8_gemm_1x128_select(null, null, null, null, null, 8, 16, 128, 2, null) == 1
     odd = ctypes.c_void_p(0x1001)
     assert lib.dg_fp8_gemm_blockscaled(odd, odd, odd, odd, odd, 8, 16, 128, null) == 3
+    # misaligned pointers are refused before any CUDA call, on every entry point
+    ok16 = ctypes.c_void_p(0x10000)
+    assert lib.dg_quantize_blockwise(odd, 8, 16, ok16, ok16, null) == 3
+    assert lib.dg_quantize_1x128(ok16, 8, 16, odd, ok16, null) == 3
+    assert lib.dg_fp8_gemm_blockscaled_bf16a(odd, ok16, ok16, ok16, ok16, ok16, 8, 16, 128, null) == 3
+    assert lib.dg_fp8_gemm_blockscaled_bf16a(ok16, ok16, ok16, ok16, odd, ok16, 8, 16, 128, null) == 3
+    assert lib.dg_fp8_gemm_1x128(ok16, ok16, odd, ok16, ok16, 8, 16, 128, null) == 3
+    assert lib.dg_fp8_grouped_gemm_contiguous(ok16, ok16, ok16, ok16, ok16, odd, 128, 2, 128, 128, null) == 3
+    assert lib.dg_fp8_grouped_gemm_masked(ok16, ok16, ok16, ok16, ok16, odd, 2, 128, 128, 128, null) == 3
+    assert lib.dg_fp8_grouped_gemm_masked(odd, ok16, ok16, ok16, ok16, ok16, 2, 128, 128, 128, null) == 3
+    # an unknown kernel choice
+    assert lib.dg_fp8_gemm_1x128_select(ok16, ok16, ok16, ok16, ok16, 8, 16, 128, 9, null) == 1
 
 
 def declared_signatures():
