@@ -104,7 +104,7 @@ using namespace dg;
 
 extern "C" {
 
-int dg_version(void) { return 100; }
+int dg_version(void) { return 101; }
 
 const char *dg_status_string(dg_status_t s) {
     switch (s) {

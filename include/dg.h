@@ -228,7 +228,8 @@ const char *dg_status_string(dg_status_t status);
  */
 dg_status_t dg_get_last_device_status(cudaStream_t stream);
 
-/* Library ABI version (major * 100 + minor). */
+/* Library ABI version (major * 100 + minor).  1.01 added the BF16-activation,
+ * per-token-scale and masked-MoE calls; every 1.00 call is unchanged. */
 int dg_version(void);
 
 /*
