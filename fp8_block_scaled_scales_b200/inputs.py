@@ -128,7 +128,7 @@ def _grouped(name, G, N, K, slots, seed, dist):
     return Grouped(name, G, N, K, counts, off, a, b, seed)
 
 
-# The five workloads (seed 1000 + workload number).
+# The workloads (seed 1000 + workload number; the masked MoE layout is number 7).
 def dense_512() -> Dense:
     """M=N=K=512, A and B from N(0,1)."""
     return _dense("dense_512", 512, 512, 512, 1001, 1.0, 1.0)
