@@ -22,7 +22,7 @@
  * Arithmetic is FP64 (see dgo_gemm_ref for why the per-K-block partial is exact).
  * Plain loops; the only parallelism is an OpenMP loop over independent rows.
  *
- * Readings where the pages are silent (each also listed in the design notes):
+ * Readings where the pages are silent:
  *   - scale s = fl32(amax / 448) by a correctly rounded division; s = 1 if amax == 0;
  *   - the quantized code is fl32(x / s) rounded to the nearest finite E4M3 value,
  *     ties to the even mantissa code, magnitudes above 448 saturate to 448, the
