@@ -18,7 +18,8 @@ LIB_PATH = os.path.join(_HERE, "libdg.so")
 
 DG_OK = 0
 STATUS_NAMES = {0: "DG_OK", 1: "DG_ERR_INVALID_ARG", 2: "DG_ERR_SHAPE", 3: "DG_ERR_ALIGNMENT",
-                4: "DG_ERR_UNSUPPORTED_DEVICE", 5: "DG_ERR_CUDA", 6: "DG_ERR_TIMEOUT"}
+                4: "DG_ERR_UNSUPPORTED_DEVICE", 5: "DG_ERR_CUDA", 6: "DG_ERR_TIMEOUT",
+                7: "DG_ERR_GROUP_OFFSETS"}
 KERNELS = {"auto": 0, "tile": 1, "skinny": 2, "pair": 3}
 
 # every symbol include/dg.h declares

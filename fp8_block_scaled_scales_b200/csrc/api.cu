@@ -13,8 +13,19 @@
 namespace dg {
 
 // The device status word: [0] status of the first failure since the last read,
-// [1] role, [2] block, [3] step.  One per device (a module global).
-__device__ int g_status[4];
+// [1] role, [2] block, [3] step; [4..7] the snapshot the last read took.  One per
+// device (a module global).
+__device__ int g_status[8];
+
+// Takes the status word: swaps [0] with zero atomically (a failure recorded
+// concurrently is kept for the next read) and copies it with its details to [4..7].
+__global__ void status_take_kernel() {
+    const int st = atomicExch(&g_status[0], 0);
+    g_status[4] = st;
+    g_status[5] = g_status[1];
+    g_status[6] = g_status[2];
+    g_status[7] = g_status[3];
+}
 
 namespace {
 
@@ -104,7 +115,7 @@ using namespace dg;
 
 extern "C" {
 
-int dg_version(void) { return 101; }
+int dg_version(void) { return 102; }
 
 const char *dg_status_string(dg_status_t s) {
     switch (s) {
@@ -115,16 +126,23 @@ const char *dg_status_string(dg_status_t s) {
         case DG_ERR_UNSUPPORTED_DEVICE: return "DG_ERR_UNSUPPORTED_DEVICE: needs compute capability 10.0 (sm_100a)";
         case DG_ERR_CUDA: return "DG_ERR_CUDA: a CUDA call failed";
         case DG_ERR_TIMEOUT: return "DG_ERR_TIMEOUT: a device pipeline wait ran past its limit";
+        case DG_ERR_GROUP_OFFSETS: return "DG_ERR_GROUP_OFFSETS: group_offsets broke its contract; nothing was computed";
     }
     return "unknown dg_status_t";
 }
 
 dg_status_t dg_get_last_device_status(cudaStream_t stream) {
-    if (cudaStreamSynchronize(stream) != cudaSuccess) return DG_ERR_CUDA;
+    DeviceInfo dev;
+    const dg_status_t st = current_device(&dev, nullptr);
+    if (st != DG_OK) return st;
+    if (cudaLaunchKernel(reinterpret_cast<const void *>(status_take_kernel), dim3(1), dim3(1), nullptr, 0,
+                         stream) != cudaSuccess)
+        return DG_ERR_CUDA;
     int h[4] = {0, 0, 0, 0};
-    if (cudaMemcpyFromSymbol(h, g_status, sizeof(h)) != cudaSuccess) return DG_ERR_CUDA;
-    const int zero[4] = {0, 0, 0, 0};
-    if (cudaMemcpyToSymbol(g_status, zero, sizeof(zero)) != cudaSuccess) return DG_ERR_CUDA;
+    if (cudaMemcpyFromSymbolAsync(h, g_status, sizeof(h), 4 * sizeof(int), cudaMemcpyDeviceToHost, stream) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
+        return DG_ERR_CUDA;
     return static_cast<dg_status_t>(h[0]);
 }
 
@@ -184,7 +202,7 @@ dg_status_t dg_fp8_gemm_blockscaled_select(const uint8_t *A, const float *sA, co
     st = current_device(&dev, nullptr);
     if (st != DG_OK) return st;
     GemmArgs a = {A, sA, B, sB, C_bf16, nullptr, M, N, K, 0};
-    if (kernel == DG_KERNEL_AUTO) kernel = M <= 128 ? DG_KERNEL_SKINNY : DG_KERNEL_PAIR;
+    if (kernel == DG_KERNEL_AUTO) kernel = M <= 128 ? DG_KERNEL_SKINNY : DG_KERNEL_TILE;
     if (kernel == DG_KERNEL_SKINNY) return launch_skinny_gemm(a, dev, stream);
     if (kernel == DG_KERNEL_TILE) return launch_tile_gemm(a, 0, dev, stream);
     return N <= 128 ? launch_pair_gemm_n128(a, dev, stream) : launch_pair_gemm(a, dev, stream);
@@ -209,7 +227,7 @@ dg_status_t dg_fp8_gemm_1x128_select(const uint8_t *A, const float *sA_t, const 
     if (st != DG_OK) return st;
     GemmArgs a = {A, sA_t, B, sB, C_bf16, nullptr, M, N, K, 0};
     a.row_scales = true;
-    if (kernel == DG_KERNEL_AUTO) kernel = M <= 128 ? DG_KERNEL_TILE : DG_KERNEL_PAIR;
+    if (kernel == DG_KERNEL_AUTO) kernel = DG_KERNEL_TILE;
     if (kernel == DG_KERNEL_TILE) return launch_tile_gemm(a, 0, dev, stream);
     return N <= 128 ? launch_pair_gemm_n128(a, dev, stream) : launch_pair_gemm(a, dev, stream);
 }

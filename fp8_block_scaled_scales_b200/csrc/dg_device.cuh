@@ -15,6 +15,7 @@ namespace dg {
 
 // Status codes written to the device status word (match dg_status_t).
 constexpr int kStatusTimeout = 6;
+constexpr int kStatusBadGroups = 7;
 
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -85,6 +86,21 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const 
     }
 }
 
+// ------------------------------------------------- programmatic dependent launch
+// The kernels are launched with programmatic stream serialisation: a kernel may
+// start while the previous kernel of the stream is still running, and runs its
+// set-up (barriers, tensor memory, descriptor and L2 prefetches) in that overlap.
+// grid_dep_wait() blocks until the previous kernel has completed and its memory is
+// visible; every thread calls it before its first global access to an input or an
+// output.  Without a programmatic predecessor it returns at once.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Lets the next kernel of the stream start its own set-up (it still waits for this
+// grid to complete before it touches memory).
+__device__ __forceinline__ void grid_dep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // --------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -99,6 +115,16 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *m
         " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
         : "memory");
+}
+
+// Prefetch one box of a 2-D tensor into L2 (no shared memory, no completion to wait
+// for).  It only warms the cache, so it may run before grid_dep_wait(): a write by
+// the previous kernel lands in L2 and a later load sees it either way.
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *map, int32_t c0, int32_t c1) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1)
+                 : "memory");
 }
 
 // 2-D tiled store shared -> global (rows/columns outside the tensor are clipped).
@@ -197,31 +223,31 @@ __device__ __forceinline__ void umma_commit(uint64_t *bar) {
                  : "memory");
 }
 
-// Load 32 consecutive FP32 columns of this warp's 32 TMEM lanes (one lane per
-// thread) and wait for the load to land.
-__device__ __forceinline__ void tmem_load32(uint32_t taddr, float (&v)[32]) {
-    uint32_t r[32];
+// Asynchronous loads of N (16, 32 or 64) consecutive FP32 columns of this warp's 32
+// TMEM lanes, one lane per thread.  The registers are written asynchronously: they
+// may only be read after tmem_wait() on the same array, which ties them so that no
+// use is hoisted above the wait.  tcgen05.wait::ld waits for every load the thread
+// has in flight.
+__device__ __forceinline__ void tmem_load_async(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
-          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
-          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr)
         : "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Issue a load of 32 consecutive FP32 columns of this warp's 32 TMEM lanes without
-// waiting.  The registers are written asynchronously: they may only be read after
-// tmem_wait32() on the same array, which ties them so that no use is hoisted above
-// the wait.
-__device__ __forceinline__ void tmem_load32_async(uint32_t taddr, uint32_t (&r)[32]) {
+__device__ __forceinline__ void tmem_wait(uint32_t (&r)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                   "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                   "+r"(r[14]), "+r"(r[15])
+                 :
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_load_async(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
         "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
@@ -235,29 +261,7 @@ __device__ __forceinline__ void tmem_load32_async(uint32_t taddr, uint32_t (&r)[
         : "memory");
 }
 
-// 16-column variant of tmem_load32_async / tmem_wait32.
-__device__ __forceinline__ void tmem_load16_async(uint32_t taddr, uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr)
-        : "memory");
-}
-
-__device__ __forceinline__ void tmem_wait16(uint32_t (&r)[16]) {
-    asm volatile("tcgen05.wait::ld.sync.aligned;"
-                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
-                   "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
-                   "+r"(r[14]), "+r"(r[15])
-                 :
-                 : "memory");
-}
-
-// Wait for every outstanding TMEM load of this thread; `r` (the most recent load's
-// destination) is tied through the wait.
-__device__ __forceinline__ void tmem_wait32(uint32_t (&r)[32]) {
+__device__ __forceinline__ void tmem_wait(uint32_t (&r)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;"
                  : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
                    "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
@@ -268,16 +272,13 @@ __device__ __forceinline__ void tmem_wait32(uint32_t (&r)[32]) {
                  : "memory");
 }
 
-// Load 64 consecutive FP32 columns of this warp's 32 TMEM lanes and wait.
-__device__ __forceinline__ void tmem_load64(uint32_t taddr, float (&v)[64]) {
-    uint32_t r[64];
+__device__ __forceinline__ void tmem_load_async(uint32_t taddr, uint32_t (&r)[64]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
         "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
         "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
         "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
-        "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
+        "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
           "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
@@ -289,8 +290,85 @@ __device__ __forceinline__ void tmem_load64(uint32_t taddr, float (&v)[64]) {
           "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
         : "r"(taddr)
         : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait(uint32_t (&r)[64]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                   "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                   "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]),
+                   "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]),
+                   "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]), "+r"(r[32]), "+r"(r[33]), "+r"(r[34]),
+                   "+r"(r[35]), "+r"(r[36]), "+r"(r[37]), "+r"(r[38]), "+r"(r[39]), "+r"(r[40]), "+r"(r[41]),
+                   "+r"(r[42]), "+r"(r[43]), "+r"(r[44]), "+r"(r[45]), "+r"(r[46]), "+r"(r[47]), "+r"(r[48]),
+                   "+r"(r[49]), "+r"(r[50]), "+r"(r[51]), "+r"(r[52]), "+r"(r[53]), "+r"(r[54]), "+r"(r[55]),
+                   "+r"(r[56]), "+r"(r[57]), "+r"(r[58]), "+r"(r[59]), "+r"(r[60]), "+r"(r[61]), "+r"(r[62]),
+                   "+r"(r[63])
+                 :
+                 : "memory");
+}
+
+// Kept for the skinny kernel: 16-column loads by the older names.
+__device__ __forceinline__ void tmem_load16_async(uint32_t taddr, uint32_t (&r)[16]) { tmem_load_async(taddr, r); }
+__device__ __forceinline__ void tmem_wait16(uint32_t (&r)[16]) { tmem_wait(r); }
+
+// Columns per TMEM load in the promotion of the tile and pair kernels.
+#ifndef DG_PROMO_CHUNK
+#define DG_PROMO_CHUNK 16
+#endif
+constexpr int kPromoChunk = DG_PROMO_CHUNK;
+
+// Promotion of one K block (the method's per-K-block scaling in FP32):
+// acc[j] += s2 * (P[2j], P[2j+1]) over the first `chunks` x CH partial-sum columns
+// (at most COLS) of this warp's 32 TMEM lanes starting at taddr, CH columns per
+// TMEM load:
+//   CH = 16 or 32: two register buffers, the load of chunk c+1 in flight while
+//                  chunk c is promoted;
+//   CH = 64:       one buffer, each load waited on before its FMAs.
+// release() runs once the last load has landed: the TMEM buffer may then be reused
+// while the last FMAs still run.
+template <int COLS, int CH, typename Release>
+__device__ __forceinline__ void promote_kblock(uint32_t taddr, float2 s2, float2 (&acc)[COLS / 2], int chunks,
+                                               Release release) {
+    static_assert(COLS % CH == 0 && (CH == 16 || CH == 32 || CH == 64), "chunk width");
+    constexpr int kChunks = COLS / CH;
+    if constexpr (CH == 64) {
 #pragma unroll
-    for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+        for (int c = 0; c < kChunks; ++c) {
+            if (c < chunks) {
+                uint32_t r[CH];
+                tmem_load_async(taddr + c * CH, r);
+                tmem_wait(r);
+                if (c + 1 == chunks) release();
+#pragma unroll
+                for (int i = 0; i < CH / 2; ++i)
+                    acc[c * (CH / 2) + i] =
+                        __ffma2_rn(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), s2,
+                                   acc[c * (CH / 2) + i]);
+            }
+        }
+    } else {
+        uint32_t r0[CH], r1[CH];
+        tmem_load_async(taddr, r0);
+        tmem_wait(r0);
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) {
+            if (c < chunks) {
+                uint32_t(&cur)[CH] = (c & 1) ? r1 : r0;
+                uint32_t(&nxt)[CH] = (c & 1) ? r0 : r1;
+                if (c + 1 < chunks)
+                    tmem_load_async(taddr + (c + 1) * CH, nxt);
+                else
+                    release();
+#pragma unroll
+                for (int i = 0; i < CH / 2; ++i)
+                    acc[c * (CH / 2) + i] =
+                        __ffma2_rn(make_float2(__uint_as_float(cur[2 * i]), __uint_as_float(cur[2 * i + 1])), s2,
+                                   acc[c * (CH / 2) + i]);
+                if (c + 1 < chunks) tmem_wait(nxt);
+            }
+        }
+    }
 }
 
 // ------------------------------------------------------- clusters and CTA pairs

@@ -34,6 +34,27 @@ struct KernelControl {
 // Valid after current_device() succeeded on the calling thread's device.
 KernelControl kernel_control();
 
+// Launches `kernel` on `stream` with programmatic stream serialisation (the kernel
+// may start its set-up while the previous kernel of the stream finishes; it calls
+// griddepcontrol.wait before touching memory).  The launch's own return code is the
+// status: an error left pending by earlier, unrelated work is neither reported as
+// this library's nor cleared.
+template <typename... KArgs, typename... Args>
+dg_status_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, size_t smem, cudaStream_t stream,
+                       Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(static_cast<unsigned>(block), 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess ? DG_OK : DG_ERR_CUDA;
+}
+
 // --- launchers (validated arguments only) ----------------------------------
 struct GemmArgs {
     const uint8_t *A;

@@ -21,8 +21,9 @@
 // Synchronisation across the pair:
 //   full[s]    even CTA only: its producer posts the byte count of both CTAs' loads,
 //              both producers' TMA loads complete on it.
-//   empty[s]   in both CTAs: each CTA's epilogue arrives once it has seen tfull for
-//              the K block that used the stage (the pair's MMAs are then done).
+//   empty[s]   in both CTAs: the MMA thread's commit (multicast) arrives on both once
+//              the pair's MMAs that read the stage are done, however far behind
+//              the epilogue runs.
 //   tfull[b]   in both CTAs: the MMA commit (multicast) arrives on both.
 // Two threads of the even CTA issue the MMAs, alternating K blocks.
 //   tempty[b]  even CTA only: all 16 epilogue warps of the pair arrive on it.
@@ -45,6 +46,8 @@ struct PairParams {
     int M, N;
     int Nb;           // ceil(N / 128)
     int Kb;           // ceil(K / 128); the last K block may be partial
+    int tiles_wide;   // tiles [0, tiles_wide) run 256 x BN; each later tile runs as two 256 x BN/2 halves
+    int num_units;    // tiles_wide + 2 * (tiles - tiles_wide)
     uint64_t timeout_ns;
     int *status;
     int debug_flags;
@@ -68,6 +71,29 @@ __device__ __forceinline__ void pair_tile_coords(int t, int num_mp, int num_n, i
     nb = local / gm;
 }
 
+// A unit of work: a whole 256 x BN tile, or (in the last round, see the launcher)
+// one 256 x BN/2 half of one.  Column n0 is the unit's first output column.
+struct PairUnit {
+    int mp;     // m-pair: rows 256 mp .. 256 mp + 255
+    int n0;     // first column
+    bool narrow;
+};
+
+template <int BN>
+__device__ __forceinline__ PairUnit pair_unit(const PairParams &p, int num_mp, int u) {
+    PairUnit w;
+    int t = u, h = 0;
+    w.narrow = u >= p.tiles_wide;
+    if (w.narrow) {
+        t = p.tiles_wide + (u - p.tiles_wide) / 2;
+        h = (u - p.tiles_wide) & 1;
+    }
+    int nb;
+    pair_tile_coords(t, num_mp, p.num_n_tiles, w.mp, nb);
+    w.n0 = nb * BN + h * (BN / 2);
+    return w;
+}
+
 template <int BN, int STAGES, int NBUF>
 struct PairSmem {
     static constexpr uint32_t kABytes = 128 * 128;
@@ -79,15 +105,15 @@ struct PairSmem {
     static constexpr uint32_t kOffBar = kOffC + 8 * kCBoxBytes;
     static constexpr uint32_t kNumBars = 2 * STAGES + 2 * NBUF + 2;
     static constexpr uint32_t kOffMisc = kOffBar + 8 * kNumBars;
-    static constexpr uint32_t kBytes = kOffMisc + 16;
+    // misc: TMEM address (0), abort flag (4); then per stage the last iteration this
+    // CTA's producer issued loads for (the leader: posted the byte count for)
+    static constexpr uint32_t kOffIssued = kOffMisc + 16;
+    static constexpr uint32_t kBytes = kOffIssued + 4 * STAGES;
     static constexpr uint32_t kDynamicBytes = kBytes + 1024;
 };
 
-// Give in-flight TMA loads time to land before a CTA that gave up leaves.
-__device__ __forceinline__ void settle_after_abort() {
-    const uint64_t t0 = globaltimer_ns();
-    while (globaltimer_ns() - t0 < 50000ull) {
-    }
+__device__ __forceinline__ void mbar_complete_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.complete_tx.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
 
 // ROWS: sA holds one scale per row of A and K block, K-block-major (sA[kb][m]);
@@ -95,11 +121,16 @@ __device__ __forceinline__ void settle_after_abort() {
 template <int BN, int STAGES, int NBUF, bool ROWS>
 __global__ void __launch_bounds__(kPairThreads, 1)
     pair_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmC, const PairParams p) {
+                     const __grid_constant__ CUtensorMap tmBn, const __grid_constant__ CUtensorMap tmC,
+                     const PairParams p) {
     using L = PairSmem<BN, STAGES, NBUF>;
-        constexpr int kColsPerWarp = BN / 2;
+    constexpr int kColsPerWarp = BN / 2;
     constexpr uint32_t kTmemCols = tmem_cols_for(NBUF * BN);
     constexpr uint32_t kIdesc = idesc_e4m3_f32(256, BN);
+    constexpr uint32_t kIdescNarrow = idesc_e4m3_f32(256, BN / 2);
+    // bytes one CTA's loads bring per K block: A + its half of the B tile
+    constexpr uint32_t kCtaBytes = L::kABytes + L::kBBytes;
+    constexpr uint32_t kCtaBytesNarrow = L::kABytes + L::kBBytes / 2;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -110,6 +141,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     uint64_t *mdone = tempty + NBUF;  // one per MMA thread: all its MMAs complete
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
+    int *issued = reinterpret_cast<int *>(smem + L::kOffIssued);
 
     const int warp = static_cast<int>(threadIdx.x >> 5);
     const int lane = lane_id();
@@ -117,11 +149,28 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const bool leader = rank == 0;
     const int pair = static_cast<int>(blockIdx.x >> 1);
     const int num_pairs = static_cast<int>(gridDim.x >> 1);
+    const int num_mp = (p.num_m + 1) / 2;
+    const int Kb = p.Kb;
+    // the units of this pair: pair, pair + num_pairs, ...
+    const int my_units = pair < p.num_units ? (p.num_units - 1 - pair) / num_pairs + 1 : 0;
+    auto unit_bytes = [&](int it) {  // one CTA's bytes in iteration `it`
+        return (pair + (it / Kb) * num_pairs) >= p.tiles_wide ? kCtaBytesNarrow : kCtaBytes;
+    };
+
+    // L2 prefetch of this CTA's first B slabs, before the dependency wait (a cache
+    // fill only, so it cannot observe stale data)
+    if (warp == 3 && lane == 0 && my_units > 0) {
+        const PairUnit w = pair_unit<BN>(p, num_mp, pair);
+        const int rows = w.narrow ? BN / 4 : BN / 2;
+        for (int kb = 0; kb < Kb && kb < 2 * STAGES; ++kb)
+            tma_prefetch_l2_2d(w.narrow ? &tmBn : &tmB, kb * 128, w.n0 + static_cast<int>(rank) * rows);
+    }
 
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
+            issued[s] = -1;
         }
         for (int q = 0; q < 2; ++q) mbar_init(&mdone[q], 1);
         for (int b = 0; b < NBUF; ++b) {
@@ -132,6 +181,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         fence_mbar_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmBn);
         tma_prefetch_desc(&tmC);
     }
     if (warp == 1) {
@@ -142,10 +192,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     cluster_sync();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-
-    const int num_mp = (p.num_m + 1) / 2;
-    const int num_tiles = num_mp * p.num_n_tiles;
-    const int Kb = p.Kb;
+    grid_dep_wait();  // inputs and outputs are touched only from here on
+    grid_dep_launch_dependents();
 
     if (warp < 4) {
         regs_dealloc<pair_regs_producer<BN>()>();
@@ -154,11 +202,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             const uint32_t full0 = mapa_shared(smem_u32(&full[0]), 0);  // the even CTA's full[0]
             int it = 0;
             bool ok = true;
-            for (int t = pair; t < num_tiles && ok; t += num_pairs) {
-                int mp, nb;
-                pair_tile_coords(t, num_mp, p.num_n_tiles, mp, nb);
-                const int a_row = (2 * mp + static_cast<int>(rank)) * 128;
-                const int b_row = nb * BN + static_cast<int>(rank) * (BN / 2);
+            for (int i = 0; i < my_units && ok; ++i) {
+                const PairUnit w = pair_unit<BN>(p, num_mp, pair + i * num_pairs);
+                const int a_row = (2 * w.mp + static_cast<int>(rank)) * 128;
+                const int b_row = w.n0 + static_cast<int>(rank) * (w.narrow ? BN / 4 : BN / 2);
                 for (int kb = 0; kb < Kb; ++kb, ++it) {
                     const int s = it % STAGES;
                     const uint32_t u = static_cast<uint32_t>(it / STAGES);
@@ -169,12 +216,13 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                         break;
                     }
                     if ((p.debug_flags & 1) && it == 0 && leader) continue;  // test hook: stage 0 never posted
-                    if (leader) mbar_arrive_expect_tx(&full[s], 2 * (L::kABytes + L::kBBytes));
+                    if (leader) mbar_arrive_expect_tx(&full[s], 2 * (w.narrow ? kCtaBytesNarrow : kCtaBytes));
+                    issued[s] = it;
                     tma_load_2d_pair(smem + L::kOffA + s * L::kABytes, &tmA, full0 + 8u * s, kb * 128, a_row);
-                    tma_load_2d_pair(smem + L::kOffB + s * L::kBBytes, &tmB, full0 + 8u * s, kb * 128, b_row);
+                    tma_load_2d_pair(smem + L::kOffB + s * L::kBBytes, w.narrow ? &tmBn : &tmB, full0 + 8u * s,
+                                     kb * 128, b_row);
                 }
             }
-            if (!ok) settle_after_abort();
         } else if ((warp == 1 || warp == 2) && lane == 0 && leader) {
             // ----------------------------------- MMA (even CTA only, two threads)
             // Thread q issues the K blocks kc with kc % 2 == q (independent partials,
@@ -182,16 +230,18 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             // buffer belongs to one thread, so its parity waits stay in order); one
             // multicast commit per K block.
             const int q = warp - 1;
-            const int my_tiles = pair < num_tiles ? (num_tiles - 1 - pair) / num_pairs + 1 : 0;
-            const int total = my_tiles * Kb;
+            const int total = my_units * Kb;
             const uint32_t a0 = smem_u32(smem + L::kOffA);
             const uint32_t b0 = smem_u32(smem + L::kOffB);
             int last = -1;
+            int unit = 0, kb = q;  // kc = unit * Kb + kb
+            while (kb >= Kb) kb -= Kb, ++unit;
             for (int kc = q; kc < total; kc += 2) {
                 const int s = kc % STAGES;
                 const uint32_t u = static_cast<uint32_t>(kc / STAGES);
                 const int buf = kc % NBUF;
                 const uint32_t v = static_cast<uint32_t>(kc / NBUF);
+                const bool narrow = pair + unit * num_pairs >= p.tiles_wide;
                 if (!mbar_wait(&tempty[buf], (v & 1u) ^ 1u, abort_flag, p.timeout_ns) ||
                     !mbar_wait(&full[s], u & 1u, abort_flag, p.timeout_ns)) {
                     record_failure(p.status, kStatusTimeout, 22, kc);
@@ -202,11 +252,15 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                 const uint64_t adesc = sdesc_kmajor_sw128(a0 + s * L::kABytes);
                 const uint64_t bdesc = sdesc_kmajor_sw128(b0 + s * L::kBBytes);
                 const uint32_t d = tmem_base + static_cast<uint32_t>(buf * BN);
+                const uint32_t idesc = narrow ? kIdescNarrow : kIdesc;
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    umma_e4m3_pair(d, adesc + 2u * k, bdesc + 2u * k, kIdesc, k > 0 ? 1u : 0u);
+                    umma_e4m3_pair(d, adesc + 2u * k, bdesc + 2u * k, idesc, k > 0 ? 1u : 0u);
+                umma_commit_pair(&empty[s], 0x3);  // both CTAs' stage s is free once these MMAs have read it
                 umma_commit_pair(&tfull[buf], 0x3);
                 last = kc;
+                kb += 2;
+                while (kb >= Kb) kb -= Kb, ++unit;
             }
             if (last >= 0) {
                 const int never = 0;
@@ -225,11 +279,12 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         float2 acc[kColsPerWarp / 2];
         int kc = 0;
         bool ok = true;
-        for (int t = pair; t < num_tiles && ok; t += num_pairs) {
-            int mp, nb;
-            pair_tile_coords(t, num_mp, p.num_n_tiles, mp, nb);
-            const int mb = 2 * mp + static_cast<int>(rank);
-            const int col0 = nb * BN + half * kColsPerWarp;
+        for (int i = 0; i < my_units && ok; ++i) {
+            const PairUnit w = pair_unit<BN>(p, num_mp, pair + i * num_pairs);
+            // this warp's columns: BN/2 of a whole tile, BN/4 of a half tile
+            const int ncols = (BN == 256 && w.narrow) ? kColsPerWarp / 2 : kColsPerWarp;
+            const int mb = 2 * w.mp + static_cast<int>(rank);
+            const int col0 = w.n0 + half * ncols;
             const int nb128 = col0 / 128;
             const bool valid = nb128 < p.Nb && mb < p.num_m;
             ScaleStream scales;
@@ -241,7 +296,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             float sa_next = row_ok ? __ldg(p.sA + my_row) : 0.0f;
             float sa_next2 = (row_ok && Kb > 1) ? __ldg(p.sA + p.M + my_row) : 0.0f;
 #pragma unroll
-            for (int i = 0; i < kColsPerWarp / 2; ++i) acc[i] = make_float2(0.0f, 0.0f);
+            for (int j = 0; j < kColsPerWarp / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
             for (int kb = 0; kb < Kb; ++kb, ++kc) {
                 const int buf = kc % NBUF;
                 const uint32_t v = static_cast<uint32_t>(kc / NBUF);
@@ -260,49 +315,32 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                     break;
                 }
                 tc_fence_after();
-                // the pair's MMAs of this K block are complete: this CTA's stage is free
-                if (ew == 0 && lane == 0) mbar_arrive(&empty[kc % STAGES]);
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                                       static_cast<uint32_t>(buf * BN + half * kColsPerWarp);
-                constexpr int kChunks = kColsPerWarp / 16;
-                uint32_t r0[16], r1[16];
-                tmem_load16_async(taddr, r0);
-                tmem_wait16(r0);
-#pragma unroll
-                for (int c = 0; c < kChunks; ++c) {
-                    uint32_t(&cur)[16] = (c & 1) ? r1 : r0;
-                    uint32_t(&nxt)[16] = (c & 1) ? r0 : r1;
-                    if (c + 1 < kChunks) {
-                        tmem_load16_async(taddr + (c + 1) * 16, nxt);
-                    } else {
-                        // this CTA's columns of the buffer are in registers: release them
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive_cluster(tempty0 + 8u * buf);
-                    }
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        acc[c * 8 + i] = __ffma2_rn(make_float2(__uint_as_float(cur[2 * i]), __uint_as_float(cur[2 * i + 1])),
-                                                    s2, acc[c * 8 + i]);
-                    if (c + 1 < kChunks) tmem_wait16(nxt);
-                }
+                                       static_cast<uint32_t>(buf * BN + half * ncols);
+                promote_kblock<kColsPerWarp, kPromoChunk>(taddr, s2, acc, ncols / kPromoChunk, [&] {
+                    // this warp's columns of the buffer are in registers: hand it back
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(tempty0 + 8u * buf);
+                });
             }
             if (!ok) break;
             const int row0 = mb * 128 + quarter * 32;
 #pragma unroll
             for (int j = 0; j < kColsPerWarp / 64; ++j) {
+                if (j * 64 >= ncols) break;
                 if (lane == 0) bulk_wait_read0();
                 __syncwarp();
                 uint8_t *rowp = cstage + lane * 128;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     const float2 *x = acc + j * 32 + c * 4;
-                    uint4 w;
-                    w.x = pack_bf16x2(x[0].x, x[0].y);
-                    w.y = pack_bf16x2(x[1].x, x[1].y);
-                    w.z = pack_bf16x2(x[2].x, x[2].y);
-                    w.w = pack_bf16x2(x[3].x, x[3].y);
-                    *reinterpret_cast<uint4 *>(rowp + ((c ^ (lane & 7)) << 4)) = w;
+                    uint4 q4;
+                    q4.x = pack_bf16x2(x[0].x, x[0].y);
+                    q4.y = pack_bf16x2(x[1].x, x[1].y);
+                    q4.z = pack_bf16x2(x[2].x, x[2].y);
+                    q4.w = pack_bf16x2(x[3].x, x[3].y);
+                    *reinterpret_cast<uint4 *>(rowp + ((c ^ (lane & 7)) << 4)) = q4;
                 }
                 fence_async_smem();
                 __syncwarp();
@@ -315,10 +353,37 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         if (lane == 0) bulk_wait_all0();
     }
 
-    // neither CTA may leave while the other can still signal its barriers or
-    // read its shared memory
+    // Neither CTA may leave while a load it issued can still land in its shared
+    // memory or signal a barrier.  Every load completes on the even CTA's full[s],
+    // whose phase for iteration `it` counts both CTAs' bytes once the even CTA has
+    // posted them.  After a normal run every posted phase has completed (the MMAs
+    // consumed them); after a timeout the even CTA drains each stage: the odd CTA's
+    // last load on a stage is either in the phase the even CTA posted last, or one
+    // phase later (it cannot run further ahead: its stage must first be freed by an
+    // MMA that waited for that phase).  Bytes that were posted but will never be sent
+    // (the odd CTA stopped first) are completed by hand; bytes sent for a phase
+    // never posted are posted now.  Every wait is bounded.
     tc_fence_before();
     __syncwarp();
+    cluster_sync();
+    if (leader && warp == 0 && lane == 0) {
+        const uint32_t peer_issued = mapa_shared(smem_u32(issued), 1);
+        const int never = 0;
+        for (int s = 0; s < STAGES; ++s) {
+            const int mine = issued[s];
+            int peer;
+            asm volatile("ld.shared::cluster.b32 %0, [%1];" : "=r"(peer) : "r"(peer_issued + 4u * s) : "memory");
+            int it = mine;
+            if (peer > mine) {
+                mbar_arrive_expect_tx(&full[s], unit_bytes(peer));  // the odd CTA's loads alone
+                it = peer;
+            } else if (mine >= 0 && peer < mine) {
+                mbar_complete_tx(&full[s], unit_bytes(mine));  // the odd CTA's share that never came
+            }
+            if (it >= 0 && !mbar_wait(&full[s], static_cast<uint32_t>(it / STAGES) & 1u, &never, p.timeout_ns))
+                record_failure(p.status, kStatusTimeout, 26, -1 - s);
+        }
+    }
     cluster_sync();
     if (warp == 1) {
         tc_fence_after();
@@ -331,11 +396,14 @@ static dg_status_t launch_pair_impl(const GemmArgs &a, const DeviceInfo &dev, cu
     using L = PairSmem<BN, STAGES, NBUF>;
     static_assert(L::kDynamicBytes <= 232448, "shared memory budget");
     static_assert(STAGES % 2 == 0 && NBUF % 2 == 0, "each MMA thread must own its stages and buffers");
-    CUtensorMap tmA, tmB, tmC;
+    CUtensorMap tmA, tmB, tmBn, tmC;
     dg_status_t st;
     st = make_tmap_2d(&tmA, a.A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.M, a.K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != DG_OK) return st;
     st = make_tmap_2d(&tmB, a.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.N, a.K, BN / 2, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != DG_OK) return st;
+    st = make_tmap_2d(&tmBn, a.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.N, a.K, BN / 4, 128,
                       CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != DG_OK) return st;
     st = make_tmap_2d(&tmC, a.C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.M, a.N, 32, 64, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -359,13 +427,15 @@ static dg_status_t launch_pair_impl(const GemmArgs &a, const DeviceInfo &dev, cu
     static thread_local int configured_device = -1;
     static thread_local int max_pairs = 0;
     int device = 0;
-    cudaGetDevice(&device);
+    if (cudaGetDevice(&device) != cudaSuccess) return DG_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.blockDim = dim3(kPairThreads, 1, 1);
     cfg.dynamicSmemBytes = L::kDynamicBytes;
     cfg.stream = stream;
@@ -385,10 +455,20 @@ static dg_status_t launch_pair_impl(const GemmArgs &a, const DeviceInfo &dev, cu
         max_pairs = clusters;
         configured_device = device;
     }
+    // Tiles go round-robin to the pairs.  When the last round would keep at most half
+    // of the pairs busy (4096^3: 256 tiles on 74 pairs leave 34 for the fourth round),
+    // its tiles run as two 256 x BN/2 halves each, so that round takes about half a
+    // tile's time; the halves are the last units, one per pair.
     const int64_t tiles = static_cast<int64_t>((p.num_m + 1) / 2) * p.num_n_tiles;
-    const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
+    if (tiles > 0x3FFFFFFFLL) return DG_ERR_SHAPE;
+    const int64_t last_round = tiles - ((tiles - 1) / max_pairs) * max_pairs;  // 1 .. max_pairs tiles
+    const bool split = BN == 256 && 2 * last_round <= max_pairs;
+    p.tiles_wide = static_cast<int>(split ? tiles - last_round : tiles);
+    p.num_units = static_cast<int>(split ? tiles + last_round : tiles);
+    const int pairs = static_cast<int>(p.num_units < max_pairs ? p.num_units : max_pairs);
     cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
-    if (cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, tmC, p) != cudaSuccess) return DG_ERR_CUDA;
+    cfg.numAttrs = 2;  // the occupancy query above ran with the cluster shape alone
+    if (cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, tmBn, tmC, p) != cudaSuccess) return DG_ERR_CUDA;
     return DG_OK;
 }
 

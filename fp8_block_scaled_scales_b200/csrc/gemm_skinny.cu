@@ -157,6 +157,12 @@ __global__ void __launch_bounds__(skinny_threads<FUSED>(), 1)
     const int kb1 = static_cast<int>((static_cast<int64_t>(p.Kb) * (rank + 1)) / S);
     const int nkb = kb1 - kb0;
 
+    // The weight slabs do not depend on the previous kernel in a decode loop, but
+    // they may; an L2 prefetch is safe either way, so it starts the weight stream
+    // before the dependency wait, overlapping the tail of the previous kernel.
+    if (warp == 2 && lane == 0)
+        for (int kb = kb0; kb < kb1; ++kb) tma_prefetch_l2_2d(&tmW, kb * 128, nb * 128);
+
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < STAGES; ++s) {
             // FUSED: a stage is full once the weight slab landed and the quantizer
@@ -187,6 +193,8 @@ __global__ void __launch_bounds__(skinny_threads<FUSED>(), 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    grid_dep_wait();  // inputs and outputs are touched only from here on
+    grid_dep_launch_dependents();
 
     if (warp == 0 && lane == 0) {
         // -------------------------------------------------------------- producer
@@ -260,6 +268,9 @@ __global__ void __launch_bounds__(skinny_threads<FUSED>(), 1)
             const uint32_t d = tmem_base + static_cast<uint32_t>(buf * MP);
 #pragma unroll
             for (int k = 0; k < 4; ++k) umma_e4m3(d, wdesc + 2u * k, xdesc + 2u * k, kIdesc, k > 0 ? 1u : 0u);
+            // unfused: the stage is free once these MMAs have read it (fused, the
+            // epilogue frees it after reading the stage's A scale)
+            if (!FUSED) umma_commit(&empty[s]);
             umma_commit(&tfull[buf]);
             last = i;
         }
@@ -365,8 +376,9 @@ __global__ void __launch_bounds__(skinny_threads<FUSED>(), 1)
                 break;
             }
             tc_fence_after();
-            // the MMAs of this K block are done: its stage may be refilled
             if (FUSED) {
+                // the MMAs of this K block are done: the stage may be refilled once
+                // every epilogue warp has read its A scale
                 // the stage's A scale, published with the stage's full phase (which
                 // is complete, and cannot advance before this warp's empty arrival)
                 const int s = i % STAGES;
@@ -378,8 +390,6 @@ __global__ void __launch_bounds__(skinny_threads<FUSED>(), 1)
                 scale = scale * sa_stage[s];  // = fl32(sA * sB), as in the unfused path
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[s]);
-            } else if (quarter == 0 && lane == 0) {
-                mbar_arrive(&empty[i % STAGES]);
             }
             const float2 s2 = make_float2(scale, scale);
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
@@ -517,13 +527,15 @@ static dg_status_t launch_skinny_impl(const GemmArgs &a, const uint16_t *Xa, uin
     cfg.blockDim = dim3(static_cast<unsigned>(skinny_threads<FUSED>()), 1, 1);
     cfg.dynamicSmemBytes = L::kDynamicBytes;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = static_cast<unsigned>(S);
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     if (cudaLaunchKernelEx(&cfg, kernel, tmW, tmX, p) != cudaSuccess) return DG_ERR_CUDA;
     return DG_OK;
 }

@@ -19,11 +19,12 @@
 //               swizzle, §4.3 multi-stage ring).
 //   warps 1-2   MMA issuers: one thread each, alternating K blocks; per K block
 //               four tcgen05.mma (K = 32 each) into that K block's TMEM partial
-//               buffer, then one commit to the buffer's "full" barrier.
+//               buffer, then a commit to the stage's "empty" barrier (the stage
+//               is free once the MMAs have read it) and one to the buffer's "full".
 //   warp 3      (kMasked) builds the m-block prefix table, then idles.
-//   warps 4-11  epilogue: per kb, free the shared-memory stage, tcgen05.ld the
-//               partial 16 columns at a time (software-pipelined against the FMAs),
-//               release the TMEM buffer as soon as the last load has landed, and
+//   warps 4-11  epilogue: per kb, tcgen05.ld the
+//               partial kPromoChunk columns at a time (promote_kblock), release
+//               the TMEM buffer as soon as the last load has landed, and
 //               acc += s * P_kb with packed FP32 FMAs (ROWS: s is the thread's
 //               row scale, loaded two K blocks ahead, times the B scale); after
 //               the last kb, round to
@@ -175,11 +176,13 @@ __device__ __forceinline__ TileInfo resolve_tile(const TileParams &p, const int 
 template <int BN, int GMODE, int STAGES, int NBUF, bool ROWS>
 __global__ void __launch_bounds__(kTileThreads, 1)
     tile_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmC, const TileParams p) {
+                     const __grid_constant__ CUtensorMap tmBn, const __grid_constant__ CUtensorMap tmC,
+                     const TileParams p) {
     using L = TileSmem<BN, STAGES, NBUF, GMODE>;
         constexpr int kColsPerWarp = BN / 2;
     constexpr uint32_t kTmemCols = tmem_cols_for(NBUF * BN);
     constexpr uint32_t kIdesc = idesc_e4m3_f32(128, BN);
+    constexpr uint32_t kIdescNarrow = idesc_e4m3_f32(128, BN / 2);
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -190,10 +193,20 @@ __global__ void __launch_bounds__(kTileThreads, 1)
     uint64_t *mdone = tempty + NBUF;  // one per MMA thread: all its MMAs complete
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
+    volatile int *groups_bad = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 8);
     int *prefix = reinterpret_cast<int *>(smem + L::kOffPrefix);  // kMasked only
 
     const int warp = static_cast<int>(threadIdx.x >> 5);
     const int lane = lane_id();
+
+    // dense: L2 prefetch of the first tile's first B slabs before the dependency
+    // wait (a cache fill only, so it cannot observe stale data); the grouped forms
+    // need the routing, an input, to know their first tile
+    if (GMODE == kDense && warp == 3 && lane == 0 && static_cast<int>(blockIdx.x) < p.num_m_cap * p.num_n_tiles) {
+        int mb, nb;
+        tile_coords(static_cast<int>(blockIdx.x), p.num_m_cap, p.num_n_tiles, mb, nb);
+        for (int kb = 0; kb < p.Kb && kb < 2 * STAGES; ++kb) tma_prefetch_l2_2d(&tmB, kb * 128, nb * BN);
+    }
 
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -206,14 +219,35 @@ __global__ void __launch_bounds__(kTileThreads, 1)
             mbar_init(&tempty[b], 8);
         }
         *abort_flag = 0;
+        *groups_bad = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmBn);
         tma_prefetch_desc(&tmC);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
+    }
+    grid_dep_wait();  // inputs and outputs are touched only from here on
+    grid_dep_launch_dependents();
+    if (GMODE == kContiguous && warp == 3) {
+        // group_offsets must start at 0, not decrease, hold multiples of 128 and end
+        // within the rows allocated; otherwise nothing is computed and the status
+        // word says why (memory stays safe either way: TMA clips every box)
+        const int cap = p.num_m_cap * 128;
+        bool bad = false;
+        for (int g = lane; g <= p.G; g += 32) {
+            const int o = __ldg(p.offsets + g);
+            const int prev = g > 0 ? __ldg(p.offsets + g - 1) : 0;
+            bad |= (o & 127) != 0 || o < prev || o > cap || (g == 0 && o != 0);
+        }
+        bad = __any_sync(0xFFFFFFFFu, bad);
+        if (lane == 0 && bad) {
+            *groups_bad = 1;
+            if (blockIdx.x == 0) record_failure(p.status, kStatusBadGroups, 3, -1);
+        }
     }
     if (GMODE == kMasked && warp == 3) {
         // prefix[g] = sum over h < g of ceil(count_h / 128): lane l takes experts
@@ -247,9 +281,36 @@ __global__ void __launch_bounds__(kTileThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    const int num_m = count_m_blocks<GMODE>(p, prefix);
+    const int num_m = (GMODE == kContiguous && *groups_bad) ? 0 : count_m_blocks<GMODE>(p, prefix);
     const int num_tiles = num_m * p.num_n_tiles;
     const int Kb = p.Kb;
+    // Tiles go round-robin to the CTAs.  When the last round would keep at most half
+    // of them busy, its tiles run as two 128 x BN/2 halves each (two units), so that
+    // round takes about half a tile's time.  Decided here because the grouped forms
+    // only know their tile count on the device; every CTA computes the same split.
+    const int grid = static_cast<int>(gridDim.x);
+    int tiles_wide = num_tiles, num_units = num_tiles;
+    if (BN == 256 && num_tiles > 0) {
+        const int last_round = num_tiles - ((num_tiles - 1) / grid) * grid;
+        if (2 * last_round <= grid) {
+            tiles_wide = num_tiles - last_round;
+            num_units = num_tiles + last_round;
+        }
+    }
+    // unit u: tile u below tiles_wide, else half (u - tiles_wide) % 2 of tile
+    // tiles_wide + (u - tiles_wide) / 2
+    auto unit_tile = [&](int u, int &t, int &h) {
+        if (u < tiles_wide) {
+            t = u;
+            h = -1;
+        } else {
+            t = tiles_wide + (u - tiles_wide) / 2;
+            h = (u - tiles_wide) & 1;
+        }
+    };
+    const int my_units = static_cast<int>(blockIdx.x) < num_units
+                             ? (num_units - 1 - static_cast<int>(blockIdx.x)) / grid + 1
+                             : 0;
 
     if (warp < 4) {
         regs_dealloc<regs_producer<BN>()>();
@@ -258,9 +319,12 @@ __global__ void __launch_bounds__(kTileThreads, 1)
             uint32_t issued = 0, parity_bits = 0;
             int it = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-                int nb;
+            for (int i = 0; i < my_units && ok; ++i) {
+                int t, h, nb;
+                unit_tile(static_cast<int>(blockIdx.x) + i * grid, t, h);
                 const TileInfo ti = resolve_tile<BN, GMODE>(p, prefix, t, num_m, nb);
+                const bool narrow = h >= 0;
+                const int b_row = ti.b_row + (narrow ? h * (BN / 2) : 0);
                 for (int kb = 0; kb < Kb; ++kb, ++it) {
                     const int s = it % STAGES;
                     const uint32_t u = static_cast<uint32_t>(it / STAGES);
@@ -271,9 +335,9 @@ __global__ void __launch_bounds__(kTileThreads, 1)
                         break;
                     }
                     if ((p.debug_flags & 1) && it == 0) continue;  // test hook: never fill stage 0
-                    mbar_arrive_expect_tx(&full[s], L::kABytes + L::kBBytes);
+                    mbar_arrive_expect_tx(&full[s], L::kABytes + (narrow ? L::kBBytes / 2 : L::kBBytes));
                     tma_load_2d(smem + L::kOffA + s * L::kABytes, &tmA, &full[s], kb * 128, ti.a_row);
-                    tma_load_2d(smem + L::kOffB + s * L::kBBytes, &tmB, &full[s], kb * 128, ti.b_row);
+                    tma_load_2d(smem + L::kOffB + s * L::kBBytes, narrow ? &tmBn : &tmB, &full[s], kb * 128, b_row);
                     issued |= 1u << s;
                     parity_bits = (parity_bits & ~(1u << s)) | ((u & 1u) << s);
                 }
@@ -291,18 +355,19 @@ __global__ void __launch_bounds__(kTileThreads, 1)
             // independent, and each issuer's barrier waits and commits hide behind the
             // other's MMAs.  With STAGES and NBUF even, every stage and every buffer
             // belongs to one thread, which therefore waits on each barrier's phases in
-            // order -- a parity wait is only sound one phase ahead.  One commit per K
-            // block: the epilogue frees the shared-memory stage once it has seen the
-            // buffer full.
+            // order -- a parity wait is only sound one phase ahead.  Two commits per K
+            // block: one frees the shared-memory stage as soon as the MMAs have read it
+            // (so the producer can refill it however far behind the epilogue runs),
+            // one marks the TMEM buffer full for the epilogue.
             const int q = warp - 1;
-            const int my_tiles = static_cast<int>(blockIdx.x) < num_tiles
-                                     ? (num_tiles - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
-                                     : 0;
-            const int total = my_tiles * Kb;
+            const int total = my_units * Kb;
             const uint32_t a0 = smem_u32(smem + L::kOffA);
             const uint32_t b0 = smem_u32(smem + L::kOffB);
             int last = -1;
+            int unit = 0, kbi = q;  // kc = unit * Kb + kbi
+            while (kbi >= Kb) kbi -= Kb, ++unit;
             for (int kc = q; kc < total; kc += 2) {
+                const bool narrow = static_cast<int>(blockIdx.x) + unit * grid >= tiles_wide;
                 const int s = kc % STAGES;
                 const uint32_t u = static_cast<uint32_t>(kc / STAGES);
                 const int buf = kc % NBUF;
@@ -317,11 +382,15 @@ __global__ void __launch_bounds__(kTileThreads, 1)
                 const uint64_t adesc = sdesc_kmajor_sw128(a0 + s * L::kABytes);
                 const uint64_t bdesc = sdesc_kmajor_sw128(b0 + s * L::kBBytes);
                 const uint32_t d = tmem_base + static_cast<uint32_t>(buf * BN);
+                const uint32_t idesc = narrow ? kIdescNarrow : kIdesc;
 #pragma unroll
                 for (int k = 0; k < 4; ++k)  // 32 bytes of K per instruction = +2 in the address field
-                    umma_e4m3(d, adesc + 2u * k, bdesc + 2u * k, kIdesc, k > 0 ? 1u : 0u);
+                    umma_e4m3(d, adesc + 2u * k, bdesc + 2u * k, idesc, k > 0 ? 1u : 0u);
+                umma_commit(&empty[s]);  // the stage is free once these MMAs have read it
                 umma_commit(&tfull[buf]);
                 last = kc;
+                kbi += 2;
+                while (kbi >= Kb) kbi -= Kb, ++unit;
             }
             // the tensor memory may only be released once every MMA issued is done
             if (last >= 0) {
@@ -340,10 +409,13 @@ __global__ void __launch_bounds__(kTileThreads, 1)
         float2 acc[kColsPerWarp / 2];
         int kc = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-            int nb;
+        for (int i = 0; i < my_units && ok; ++i) {
+            int t, h, nb;
+            unit_tile(static_cast<int>(blockIdx.x) + i * grid, t, h);
             const TileInfo ti = resolve_tile<BN, GMODE>(p, prefix, t, num_m, nb);
-            const int col0 = nb * BN + half * kColsPerWarp;
+            // this warp's columns: BN/2 of a whole tile, BN/4 of a half tile
+            const int ncols = h >= 0 ? kColsPerWarp / 2 : kColsPerWarp;
+            const int col0 = nb * BN + (h >= 0 ? h * (BN / 2) : 0) + half * ncols;
             const int nb128 = col0 / 128;
             const bool n_valid = nb128 < p.Nb;
             const int sb_row = ti.sb_row + nb128;
@@ -375,40 +447,22 @@ __global__ void __launch_bounds__(kTileThreads, 1)
                     break;
                 }
                 tc_fence_after();
-                // the MMAs of this K block are complete, so its shared-memory stage is free
-                if (ew == 0 && lane == 0) mbar_arrive(&empty[kc % STAGES]);
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                                       static_cast<uint32_t>(buf * BN + half * kColsPerWarp);
-                // 16 columns at a time: the load of chunk c+1 is in flight while chunk c
-                // is promoted; the buffer is handed back as soon as the last load landed.
-                constexpr int kChunks = kColsPerWarp / 16;
-                uint32_t r0[16], r1[16];
-                tmem_load16_async(taddr, r0);
-                tmem_wait16(r0);
-#pragma unroll
-                for (int c = 0; c < kChunks; ++c) {
-                    uint32_t(&cur)[16] = (c & 1) ? r1 : r0;
-                    uint32_t(&nxt)[16] = (c & 1) ? r0 : r1;
-                    if (c + 1 < kChunks) {
-                        tmem_load16_async(taddr + (c + 1) * 16, nxt);
-                    } else {
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&tempty[buf]);
-                    }
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        acc[c * 8 + i] = __ffma2_rn(make_float2(__uint_as_float(cur[2 * i]), __uint_as_float(cur[2 * i + 1])),
-                                                    s2, acc[c * 8 + i]);
-                    if (c + 1 < kChunks) tmem_wait16(nxt);
-                }
+                                       static_cast<uint32_t>(buf * BN + half * ncols);
+                promote_kblock<kColsPerWarp, kPromoChunk>(taddr, s2, acc, ncols / kPromoChunk, [&] {
+                    // this warp's columns of the buffer are in registers: hand it back
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&tempty[buf]);
+                });
             }
             if (!ok) break;
-            // BF16 output: rows a_row + 32*quarter + lane, columns col0 .. col0 + kColsPerWarp
+            // BF16 output: rows a_row + 32*quarter + lane, columns col0 .. col0 + ncols
             const int row0 = ti.a_row + quarter * 32;
             const int vrows = ti.rows - quarter * 32;  // rows of this warp's box that hold output
 #pragma unroll
             for (int j = 0; j < kColsPerWarp / 64; ++j) {
+                if (j * 64 >= ncols) break;
                 if (GMODE == kMasked && vrows < 32) {
                     // the box runs past the expert's tokens: each row that holds
                     // output stores itself, the rest of the slab is left untouched
@@ -461,13 +515,16 @@ static dg_status_t launch_tile_impl(const GemmArgs &a, const DeviceInfo &dev, cu
     using L = TileSmem<BN, STAGES, NBUF, GMODE>;
     static_assert(L::kDynamicBytes <= 232448, "shared memory budget");
     static_assert(STAGES % 2 == 0 && NBUF % 2 == 0, "each MMA thread must own its stages and buffers");
-    CUtensorMap tmA, tmB, tmC;
+    CUtensorMap tmA, tmB, tmBn, tmC;
     const uint64_t b_rows = GMODE != kDense ? static_cast<uint64_t>(a.G) * a.N : static_cast<uint64_t>(a.N);
     dg_status_t st;
     st = make_tmap_2d(&tmA, a.A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.M, a.K, 128, 128,
                       CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != DG_OK) return st;
     st = make_tmap_2d(&tmB, a.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, b_rows, a.K, BN, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != DG_OK) return st;
+    st = make_tmap_2d(&tmBn, a.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, b_rows, a.K, BN / 2, 128,
                       CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != DG_OK) return st;
     st = make_tmap_2d(&tmC, a.C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.M, a.N, 32, 64,
@@ -511,9 +568,11 @@ static dg_status_t launch_tile_impl(const GemmArgs &a, const DeviceInfo &dev, cu
     // kMasked: the counts live on the device, so size the grid for full slabs
     const int64_t m_blocks = GMODE == kMasked ? static_cast<int64_t>(a.G) * p.mb_max : p.num_m_cap;
     const int64_t tiles = m_blocks * p.num_n_tiles;
-    const int grid = static_cast<int>(tiles < dev.num_sms ? tiles : dev.num_sms);
-    kernel<<<grid, kTileThreads, L::kDynamicBytes, stream>>>(tmA, tmB, tmC, p);
-    return cudaGetLastError() == cudaSuccess ? DG_OK : DG_ERR_CUDA;
+    if (tiles > 0x3FFFFFFFLL) return DG_ERR_SHAPE;
+    // up to twice the tiles: a single partial round may run as half tiles (see the kernel)
+    const int64_t want = BN == 256 ? 2 * tiles : tiles;
+    const int grid = static_cast<int>(want < dev.num_sms ? want : dev.num_sms);
+    return launch_pdl(kernel, grid, kTileThreads, L::kDynamicBytes, stream, tmA, tmB, tmBn, tmC, p);
 }
 
 dg_status_t launch_tile_gemm(const GemmArgs &a, int group, const DeviceInfo &dev, cudaStream_t stream) {

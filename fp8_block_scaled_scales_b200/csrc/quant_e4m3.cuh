@@ -6,11 +6,9 @@
 // Division: fl32(x/s) is needed only through its E4M3 rounding.  The code forms
 // y = x * r with r = 1/s correctly rounded (__frcp_rn).  Two roundings of relative
 // size <= 2^-24 each put y within 2 FP32 ulps of x/s, and fl32(x/s) is within half
-// an ulp of it; so unless y lies within a few ulps of an E4M3 rounding midpoint
-// (mantissa pattern ...1000...0 at the 4th bit), y and fl32(x/s) round to the same
-// E4M3 code.  Near a midpoint, below the E4M3 normal range (where the midpoints
-// sit at other bit positions) or when r is not finite, the IEEE division x / s is
-// used instead.
+// an ulp of it; so unless an E4M3 rounding boundary lies within 3 ulps of y, y and
+// fl32(x/s) round to the same E4M3 code.  Near a boundary (see quantize8) or when
+// r is not finite, the IEEE division x / s is used instead.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -65,27 +63,42 @@ __device__ __forceinline__ BlockScale block_scale(uint32_t amax_bits) {
 
 // Eight BF16 (one 16-byte group) -> eight E4M3 codes.
 //
-// y = x * r decides the same code as fl32(x / s) unless y lies within a few FP32
-// ulps of an E4M3 rounding midpoint (mantissa bit 19 set and bits 0-18 clear:
-// bits[19:0] in [0x7FFFA, 0x80006]) or below 2^-6, where E4M3 is subnormal and its
-// midpoints sit at other bit positions.  Both conditions are tracked branch-free
-// as running minima over the eight values (distance to the midpoint pattern, and
-// |y|); only when one fires -- rarely -- are the eight quotients recomputed with
-// IEEE division.
+// y = x * r is within 3 FP32 ulps of fl32(x / s), so the two round to the same E4M3
+// code unless an E4M3 rounding boundary lies within 3 ulps of y.  Two screens find
+// every such y, branch-free, over the eight values:
+//   - normal range (|y| >= 2^-6): the boundaries are the FP32 values whose mantissa
+//     is ...1000...0 below the three kept bits, i.e. bits[19:0] == 0x80000; y is
+//     within 6 ulps of one iff (bits + 0x80006) & 0xFFFFF <= 12;
+//   - below 2^-6 (E4M3 subnormals, quantum 2^-9): the boundaries are the odd
+//     multiples of 2^-10, i.e. 1024 y an odd integer.  With M = 1.5 * 2^23,
+//     rr = fl32(1024 y + M) holds the nearest integer n to 1024 y in its last bits
+//     (its lowest bit is n's parity), and d = 1024 y - n is exact; 3 ulps of y
+//     below 2^-6 are at most 3 * 2^-20 in these units, so the test is |d| <= 2^-18
+//     with n odd.  Values that are exact E4M3 numbers (n even), zero included, never
+//     fire.
+// Only when a screen fires -- about once in 10^5 values -- are the eight quotients
+// recomputed with IEEE division.  (A screen that sent every |y| < 2^-6 to the
+// division fired in most warps: measured, half the quantizer's time.)
 __device__ __forceinline__ uint2 quantize8(uint4 v, const BlockScale &b) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    const float2 k1024 = make_float2(1024.0f, 1024.0f);
+    const float2 magic = make_float2(0x1.8p23f, 0x1.8p23f);
+    const float2 neg_magic = make_float2(-0x1.8p23f, -0x1.8p23f);
     float2 x[4], y[4];
-    uint32_t dmin = 0xFFFFFFFFu;
-    float ymin = 1.0f;
+    uint32_t dmin = 0xFFFFFFFFu, sub = 0;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         x[j] = make_float2(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xFFFF0000u));
         y[j] = __fmul2_rn(x[j], b.r2);
         dmin = min(dmin, (__float_as_uint(y[j].x) + 0x80006u) & 0xFFFFFu);
         dmin = min(dmin, (__float_as_uint(y[j].y) + 0x80006u) & 0xFFFFFu);
-        ymin = fminf(ymin, fminf(fabsf(y[j].x), fabsf(y[j].y)));
+        const float2 rr = __ffma2_rn(y[j], k1024, magic);
+        const float2 n = __fadd2_rn(rr, neg_magic);
+        const float2 d = __ffma2_rn(y[j], k1024, make_float2(-n.x, -n.y));
+        sub |= (fabsf(d.x) <= 0x1p-18f) ? (__float_as_uint(rr.x) & 1u) : 0u;
+        sub |= (fabsf(d.y) <= 0x1p-18f) ? (__float_as_uint(rr.y) & 1u) : 0u;
     }
-    if (__builtin_expect(dmin <= 12u || ymin < 0x1p-6f || !b.fast_ok, 0)) {
+    if (__builtin_expect(dmin <= 12u || sub != 0u || !b.fast_ok, 0)) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) y[j] = make_float2(__fdiv_rn(x[j].x, b.s), __fdiv_rn(x[j].y, b.s));
     }

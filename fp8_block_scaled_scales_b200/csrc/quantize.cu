@@ -29,6 +29,8 @@ __global__ void __launch_bounds__(kQuantThreads)
     quantize_kernel(const uint16_t *__restrict__ X, int64_t R, int64_t C, int64_t Cb, uint8_t *__restrict__ Q,
                     float *__restrict__ S) {
     __shared__ uint32_t red[kQuantThreads / 32];
+    grid_dep_wait();  // X may come from the previous kernel
+    grid_dep_launch_dependents();
     const int64_t blk = blockIdx.x;
     const int64_t br = blk / Cb, bc = blk - br * Cb;
     const int tid = static_cast<int>(threadIdx.x);
@@ -80,6 +82,8 @@ __global__ void __launch_bounds__(kQuantThreads)
 __global__ void __launch_bounds__(kQuantThreads)
     quantize_groups_kernel(const uint16_t *__restrict__ X, int64_t R, int64_t C, int64_t Cb, int64_t groups,
                            uint8_t *__restrict__ Q, float *__restrict__ St) {
+    grid_dep_wait();  // X may come from the previous kernel
+    grid_dep_launch_dependents();
     const int tid = static_cast<int>(threadIdx.x);
     const int64_t gi = static_cast<int64_t>(blockIdx.x) * (kQuantThreads / 16) + (tid >> 4);
     const bool group_ok = gi < groups;
@@ -103,9 +107,8 @@ dg_status_t launch_quantize_groups(const void *X, int64_t rows, int64_t cols, ui
     const int64_t groups = rows * Cb;
     const int64_t blocks = (groups + kQuantThreads / 16 - 1) / (kQuantThreads / 16);
     if (blocks > 0x7FFFFFFFLL) return DG_ERR_SHAPE;
-    quantize_groups_kernel<<<static_cast<unsigned>(blocks), kQuantThreads, 0, stream>>>(
-        static_cast<const uint16_t *>(X), rows, cols, Cb, groups, Q, St);
-    return cudaGetLastError() == cudaSuccess ? DG_OK : DG_ERR_CUDA;
+    return launch_pdl(quantize_groups_kernel, static_cast<int>(blocks), kQuantThreads, 0, stream,
+                      static_cast<const uint16_t *>(X), rows, cols, Cb, groups, Q, St);
 }
 
 dg_status_t launch_quantize(const void *X, int64_t rows, int64_t cols, uint8_t *Q, float *S,
@@ -114,9 +117,8 @@ dg_status_t launch_quantize(const void *X, int64_t rows, int64_t cols, uint8_t *
     const int64_t Rb = (rows + 127) / 128, Cb = (cols + 127) / 128;
     const int64_t blocks = Rb * Cb;
     if (blocks > 0x7FFFFFFFLL) return DG_ERR_SHAPE;
-    quantize_kernel<<<static_cast<unsigned>(blocks), kQuantThreads, 0, stream>>>(
-        static_cast<const uint16_t *>(X), rows, cols, Cb, Q, S);
-    return cudaGetLastError() == cudaSuccess ? DG_OK : DG_ERR_CUDA;
+    return launch_pdl(quantize_kernel, static_cast<int>(blocks), kQuantThreads, 0, stream,
+                      static_cast<const uint16_t *>(X), rows, cols, Cb, Q, S);
 }
 
 }  // namespace dg

@@ -37,6 +37,15 @@
  *     DG_ERR_UNSUPPORTED_DEVICE.  There is no fallback path.
  *   - Calls that overlap on the GPU are independent unless they write the same
  *     output.  Results are bitwise run-to-run deterministic.
+ *   - Kernels are launched with programmatic stream serialisation: a kernel may
+ *     start its set-up (barriers, tensor memory, descriptor and L2 prefetches of
+ *     weights) while the previous kernel on `stream` finishes, and waits for that
+ *     kernel to complete before it reads or writes any argument.  Stream order is
+ *     unchanged.
+ *   - Resources: the library allocates no device memory.  Its per-device state is
+ *     a small status word in the module's global memory plus host-side caches of
+ *     device attributes; they live until the process exits, so there is no
+ *     initialisation or shutdown call.
  */
 #ifndef DG_H_
 #define DG_H_
@@ -55,7 +64,8 @@ typedef enum {
     DG_ERR_ALIGNMENT = 3,          /* a pointer not aligned as required */
     DG_ERR_UNSUPPORTED_DEVICE = 4, /* current device is not compute capability 10.0 */
     DG_ERR_CUDA = 5,               /* a CUDA runtime/driver call failed */
-    DG_ERR_TIMEOUT = 6             /* device: a pipeline wait ran past its limit */
+    DG_ERR_TIMEOUT = 6,            /* device: a pipeline wait ran past its limit */
+    DG_ERR_GROUP_OFFSETS = 7       /* device: group_offsets broke its contract; nothing was computed */
 } dg_status_t;
 
 /*
@@ -91,7 +101,9 @@ dg_status_t dg_quantize_blockwise(const void *X_bf16, int64_t rows, int64_t cols
  * dg_quantize_blockwise produces them (each K step clipped to what remains,
  * demingchina.com/news/60142 §6.3).
  * M == 0 or N == 0 is a no-op.  M <= 128 takes the skinny split-K kernel,
- * larger M the persistent CTA-pair tile kernel; both compute the same formula.
+ * larger M the persistent single-CTA tile kernel (128 x 256 tiles; a last round
+ * of tiles that would leave at least half the SMs idle runs as 128 x 128 halves);
+ * both compute the same formula.
  */
 dg_status_t dg_fp8_gemm_blockscaled(const uint8_t *A, const float *sA,
                                     const uint8_t *B, const float *sB, void *C_bf16,
@@ -135,6 +147,10 @@ dg_status_t dg_fp8_gemm_blockscaled_bf16a(const void *A_bf16, const uint8_t *B, 
  * group_offsets : DEVICE int32 [G+1], off[0] == 0, non-decreasing, each a
  *                 multiple of 128, off[G] <= M_total_capacity.  Read on the
  *                 device, so it may be produced by an earlier kernel on `stream`.
+ *                 The kernel checks these rules before it computes anything; an
+ *                 array that breaks one leaves C untouched and records
+ *                 DG_ERR_GROUP_OFFSETS in the device status word
+ *                 (dg_get_last_device_status); the call itself returns DG_OK.
  * M_total_capacity % 128 == 0, 1 <= G <= 1024, N % 128 == 0, K % 16 == 0, K > 0
  * (a partial last K block as in dg_fp8_gemm_blockscaled).
  * M_total_capacity == 0 or N == 0 is a no-op.
@@ -168,7 +184,7 @@ dg_status_t dg_quantize_1x128(const void *X_bf16, int64_t rows, int64_t cols,
  *
  * A    : [M][K] E4M3.            sA_t : [ceil(K/128)][M] FP32 (from dg_quantize_1x128).
  * B, sB, C and the shape rules as in dg_fp8_gemm_blockscaled.
- * M <= 128 runs the tile kernel, larger M the CTA-pair kernel.
+ * Runs the single-CTA tile kernel.
  */
 dg_status_t dg_fp8_gemm_1x128(const uint8_t *A, const float *sA_t,
                               const uint8_t *B, const float *sB, void *C_bf16,
@@ -199,10 +215,12 @@ dg_status_t dg_fp8_grouped_gemm_masked(const uint8_t *A, const float *sA,
 
 /*
  * Kernel selection for the dense GEMM, for tests and measurement.  AUTO is the
- * dispatch dg_fp8_gemm_blockscaled uses: SKINNY for M <= 128, else PAIR.
+ * dispatch dg_fp8_gemm_blockscaled uses: SKINNY for M <= 128, else TILE.
  *   TILE    persistent single-CTA kernel, 128 x 256 (128 x 128 if N <= 128) tiles;
  *   SKINNY  split-K kernel for M <= 128 (larger M gives DG_ERR_SHAPE);
  *   PAIR    persistent CTA-pair kernel, 256 x 256 (256 x 128 if N <= 128) tiles.
+ * TILE and PAIR run a last round that would leave at least half the SMs idle as
+ * half-width tiles.
  */
 typedef enum { DG_KERNEL_AUTO = 0, DG_KERNEL_TILE = 1, DG_KERNEL_SKINNY = 2, DG_KERNEL_PAIR = 3 } dg_kernel_t;
 
@@ -222,24 +240,28 @@ dg_status_t dg_fp8_gemm_1x128_select(const uint8_t *A, const float *sA_t,
 const char *dg_status_string(dg_status_t status);
 
 /*
- * Synchronises `stream`, returns the device status word recorded by kernels of
- * this library on the current device since the previous call (DG_OK if none),
- * and clears it.
+ * Returns the device status word recorded by kernels of this library on the
+ * current device since the previous call (DG_OK if none) and clears it: a small
+ * kernel on `stream` swaps the word with zero atomically, so a failure recorded
+ * concurrently is kept for the next call, not lost; then `stream` is
+ * synchronised.  Failures of kernels on other streams are covered once those
+ * kernels have completed (synchronise them first).
  */
 dg_status_t dg_get_last_device_status(cudaStream_t stream);
 
 /* Library ABI version (major * 100 + minor).  1.01 added the BF16-activation,
- * per-token-scale and masked-MoE calls; every 1.00 call is unchanged. */
+ * per-token-scale and masked-MoE calls; 1.02 added DG_ERR_GROUP_OFFSETS.  Every
+ * 1.00 call is unchanged. */
 int dg_version(void);
 
 /*
  * Test-only control of the kernels' failure detection.  Every wait inside the
  * kernels gives up after timeout_ns nanoseconds (0 restores the default of 2 s),
  * records DG_ERR_TIMEOUT in the device status word and lets the kernel finish
- * cleanly.  debug_flags bit 0 makes the tile kernel's TMA producer skip its first
- * shared-memory stage, so that the MMA warp's wait runs out: it exercises the
- * timeout path without faulting or hanging the GPU.  Applies to launches made
- * after the call, process-wide; not for production use.
+ * cleanly.  debug_flags bit 0 makes the TMA producer of the tile, pair and skinny
+ * kernels skip its first shared-memory stage, so that the MMA warp's wait runs
+ * out: it exercises the timeout path without faulting or hanging the GPU.
+ * Applies to launches made after the call, process-wide; not for production use.
  */
 void dg_test_set_kernel_control(uint64_t timeout_ns, int debug_flags);
 

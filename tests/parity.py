@@ -35,3 +35,28 @@ def stratified_rms(ref_rows: np.ndarray, row_weights: np.ndarray) -> float:
     """RMS over all rows of a matrix from a weighted sample of its rows."""
     ms = np.mean(ref_rows * ref_rows, axis=1)
     return float(np.sqrt(np.sum(ms * row_weights) / np.sum(row_weights)))
+
+
+def grouped_ref_rows(qa, sa, qb, sb, offsets, rows):
+    """Oracle values of the grouped-contiguous layout at `rows` (all columns), one
+    dense oracle call per expert on the expert's slice: the grouped form is the dense
+    formula per expert (pinned in the oracle tests), and the dense routine decodes
+    each expert's weights once instead of once per row."""
+    rows = np.asarray(rows, dtype=np.int64)
+    out = np.full((rows.size, qb.shape[1]), np.nan)
+    owner = np.searchsorted(offsets, rows, side="right") - 1
+    for g in np.unique(owner):
+        sel = np.flatnonzero(owner == g)
+        r0, r1 = int(offsets[g]), int(offsets[g + 1])
+        out[sel] = oracle.gemm_ref(qa[r0:r1], sa[r0 // 128:r1 // 128], qb[g], sb[g], rows=rows[sel] - r0)
+    return out
+
+
+def rows_per_quarter(first: int, count: int, rng) -> list:
+    """One random row in each 32-row quarter of the 128-row block at `first` that
+    holds any of the block's first `count` rows: every epilogue warp's output of
+    every tile of that block is then checked."""
+    rows = []
+    for q0 in range(0, min(count, 128), 32):
+        rows.append(first + q0 + int(rng.integers(0, min(32, count - q0))))
+    return rows

@@ -38,9 +38,13 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.dg_version() == 101
+    assert lib.dg_version() == 102
     for code, name in binding.STATUS_NAMES.items():
         assert lib.dg_status_string(code).decode().startswith(name)
+    # the device-side group_offsets check has its own code, named in the header
+    assert binding.STATUS_NAMES[7] == "DG_ERR_GROUP_OFFSETS"
+    with open(os.path.join(ROOT, "include", "dg.h")) as f:
+        assert "DG_ERR_GROUP_OFFSETS = 7" in f.read()
 
 
 def test_host_validation_without_device(lib):

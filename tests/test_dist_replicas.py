@@ -50,12 +50,12 @@ def test_reference_arm_prints_on_rank0_only(tmp_path):
     import subprocess
     env = dict(os.environ, WORLD_SIZE="2", RANK="1", LOCAL_RANK="1", CUDA_VISIBLE_DEVICES="")
     p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
-                        "--warmup", "0", "--workload", "dense_512", "--oracle-rows", "8"],
+                        "--warmup", "0", "--workload", "dense_512", "--oracle-gflop", "0.02"],
                        env=env, capture_output=True, text=True, timeout=300)
     assert p.returncode == 0 and p.stdout.strip() == ""
     env["RANK"], env["LOCAL_RANK"] = "0", "0"
     p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
-                        "--warmup", "0", "--workload", "dense_512", "--oracle-rows", "8"],
+                        "--warmup", "0", "--workload", "dense_512", "--oracle-gflop", "0.02"],
                        env=env, capture_output=True, text=True, timeout=300)
     assert p.returncode == 0
     line = json.loads(p.stdout.strip().splitlines()[-1])

@@ -1,7 +1,8 @@
 """GPU parity of the dense block-scaled GEMM against the oracle, element by element.
 
-Small shapes are compared in full (several tiles and ragged tails); the full-size
-workloads on sampled rows.  Tolerance: |c - ref| <= 1e-2 |ref| + 1e-3 rms(ref).
+Small shapes and the 4096^3 workload are compared in full (several tiles and ragged
+tails); 8192^3 on one row in every 32-row quarter of every 128-row block (every tile
+and every epilogue warp's share of it).  Tolerance: |c - ref| <= 1e-2 |ref| + 1e-3 rms(ref).
 """
 import numpy as np
 import pytest
@@ -10,7 +11,7 @@ import torch
 import oracle
 from fp8_block_scaled_scales_b200 import binding, inputs
 
-from parity import c_f64, check, dev, oracle_quant, stratified_rms
+from parity import c_f64, check, dev, oracle_quant, rows_per_quarter, stratified_rms
 
 pytestmark = pytest.mark.gpu
 
@@ -147,15 +148,18 @@ def test_dense_unit_scale_identity_invariant():
 
 
 # ---------------------------------------------------------------- full-size workloads
-def _sampled_rows_check(d, kernel="auto", n_random=48, seed=0):
+def _every_tile_check(d, kernel="auto", seed=0):
+    """One row in every 32-row quarter of every 128-row block, all columns, plus the
+    outlier rows and the edges: every tile (and each epilogue warp's share of it) of
+    the persistent schedule, whichever wave or raster group it fell in, is compared."""
     qa, sa, qb, sb = quantized(d)
     c = c_f64(run(qa, sa, qb, sb, kernel=kernel))
     rng = np.random.default_rng(seed)
+    picks = []
+    for b in range(0, d.M, 128):
+        picks += rows_per_quarter(b, d.M - b, rng)
     special = set(d.outliers.tolist())
-    normal = np.array(sorted(set(range(d.M)) - special))
-    picks = rng.choice(normal, size=min(n_random, normal.size), replace=False)
-    edges = [0, d.M - 1, min(127, d.M - 1), min(128, d.M - 1)]
-    rows = np.unique(np.concatenate([picks, list(special), edges]).astype(np.int64))
+    rows = np.unique(np.concatenate([picks, list(special), [0, d.M - 1]]).astype(np.int64))
     ref = oracle.gemm_ref(qa, sa, qb, sb, rows=rows)
     is_out = np.isin(rows, d.outliers)
     w = np.where(is_out, len(special) / max(is_out.sum(), 1), (d.M - len(special)) / max((~is_out).sum(), 1))
@@ -164,7 +168,11 @@ def _sampled_rows_check(d, kernel="auto", n_random=48, seed=0):
 
 
 def test_dense_4096_outliers_workload():
-    _sampled_rows_check(inputs.dense_4096_outliers())
+    """The headline workload compared in full: all 4096 x 4096 outputs."""
+    d = inputs.dense_4096_outliers()
+    qa, sa, qb, sb = quantized(d)
+    c = c_f64(run(qa, sa, qb, sb))
+    check(c, oracle.gemm_ref(qa, sa, qb, sb), None, d.name)
 
 
 @pytest.mark.parametrize("M", [1, 16, 64, 128])
@@ -178,7 +186,7 @@ def test_skinny_workload(M):
 
 @pytest.mark.slow
 def test_dense_8192_workload():
-    _sampled_rows_check(inputs.dense_8192(), n_random=24)
+    _every_tile_check(inputs.dense_8192())
 
 
 @pytest.mark.parametrize("M,N,K,kernel", [(512, 768, 1024, "pair"), (512, 768, 1024, "tile"),

@@ -6,7 +6,7 @@ import torch
 import oracle
 from fp8_block_scaled_scales_b200 import binding, inputs
 
-from parity import c_f64, check, dev, oracle_quant, stratified_rms
+from parity import c_f64, check, dev, grouped_ref_rows, oracle_quant, rows_per_quarter
 
 pytestmark = pytest.mark.gpu
 
@@ -82,29 +82,69 @@ def test_grouped_offsets_read_on_device():
     check(c_f64(C)[real], ref[real], float(np.sqrt(np.mean(ref[real] ** 2))), "device offsets")
 
 
-def _grouped_workload_check(w, per_expert_rows=2, n_random=64, seed=0):
+def _grouped_workload_check(w, full=False, seed=0):
+    """All real rows (full), or one real row in every 32-row quarter of every 128-row
+    block that holds tokens plus each expert's first and last real row: every tile
+    of the schedule is compared either way.  Padding rows must be exactly zero."""
     qa, sa, qb, sb = quantized(w)
     C = run(qa, sa, qb, sb, w.offsets)
     c = c_f64(C)
-    rng = np.random.default_rng(seed)
     real = inputs.real_row_mask(w.counts, w.offsets)
-    real_rows = np.flatnonzero(real)
-    rows = set(rng.choice(real_rows, size=n_random, replace=False).tolist())
-    for g in range(w.G):  # each expert's first and last real row
-        if w.counts[g]:
-            rows.add(int(w.offsets[g]))
-            rows.add(int(w.offsets[g] + w.counts[g] - 1))
-    rows = np.array(sorted(rows), dtype=np.int64)
-    ref = oracle.grouped_gemm_ref(qa, sa, qb, sb, w.offsets, rows)
+    if full:
+        rows = np.flatnonzero(real)
+    else:
+        rng = np.random.default_rng(seed)
+        rows = set()
+        for g in range(w.G):
+            n = int(w.counts[g])
+            if not n:
+                continue
+            r0 = int(w.offsets[g])
+            rows.update([r0, r0 + n - 1])
+            for b in range(0, n, 128):
+                rows.update(rows_per_quarter(r0 + b, n - b, rng))
+        rows = np.array(sorted(rows), dtype=np.int64)
+    ref = grouped_ref_rows(qa, sa, qb, sb, w.offsets, rows)
     rms = float(np.sqrt(np.mean(ref ** 2)))
     check(c[rows], ref, rms, w.name)
     assert np.all(c[~real] == 0.0)
 
 
 def test_moe_g8_workload():
-    _grouped_workload_check(inputs.moe_g8())
+    """Every real row of the 8-expert workload (16384 token slots x 4096 columns)."""
+    _grouped_workload_check(inputs.moe_g8(), full=True)
 
 
 @pytest.mark.slow
 def test_moe_g64_zipf_workload():
-    _grouped_workload_check(inputs.moe_g64_zipf(), n_random=32)
+    _grouped_workload_check(inputs.moe_g64_zipf())
+
+
+@pytest.mark.parametrize("bad", ["not_a_multiple_of_128", "decreasing", "past_capacity", "nonzero_start"])
+def test_grouped_malformed_offsets_leave_c_untouched_and_set_status(bad):
+    """group_offsets that break their contract: the kernel computes nothing, records
+    DG_ERR_GROUP_OFFSETS in the device status word (no trap, the context stays
+    usable) and a correct call afterwards computes normally."""
+    counts = [128, 256, 0, 100]
+    w = inputs.grouped_custom(4, 256, 256, counts, seed=9300)
+    qa, sa, qb, sb = quantized(w)
+    off = w.offsets.copy()  # [0, 128, 384, 384, 512]
+    cap = int(off[-1])
+    if bad == "not_a_multiple_of_128":
+        off[2] = 300
+    elif bad == "decreasing":
+        off[2] = 100
+    elif bad == "past_capacity":
+        off[4] = cap + 128
+    else:
+        off[0] = 128
+    C = torch.full((cap, 256), -5.0, dtype=torch.bfloat16, device="cuda")
+    binding.grouped_gemm_contiguous(dev(qa), dev(sa), dev(qb), dev(sb), dev(off), C=C)
+    torch.cuda.synchronize()
+    assert binding.last_device_status() == 7
+    assert torch.all(C == -5.0)
+    assert binding.last_device_status() == 0  # the read cleared it
+    C2 = run(qa, sa, qb, sb, w.offsets)
+    ref = oracle.grouped_gemm_ref(qa, sa, qb, sb, w.offsets, np.arange(cap))
+    real = inputs.real_row_mask(w.counts, w.offsets)
+    check(c_f64(C2)[real], ref[real], float(np.sqrt(np.mean(ref[real] ** 2))), "after a malformed call")

@@ -61,6 +61,43 @@ def test_quantize_rounding_boundaries():
     run_and_compare(y)
 
 
+def _bf16_from_bits(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(bits.astype(np.uint16).view(np.int16)).view(torch.bfloat16)
+
+
+def test_quantize_every_bf16_pattern_under_a_scale_sweep():
+    """Every finite BF16 value, under block scales that are powers of two (x/s then
+    lands exactly on E4M3 values, midpoints and their neighbours), one BF16 step above
+    and below them, and a few arbitrary ones: the codes and scales must equal the
+    oracle's (which divides in FP64 and rounds once) bit for bit.  Each 128x128 block
+    holds the patterns not larger than its amax plus one element equal to it."""
+    pos = np.arange(0x0000, 0x7F80, dtype=np.uint32)            # +0 .. largest finite
+    bits = np.concatenate([pos, pos | 0x8000])                    # and their negatives
+    mag = (pos.astype(np.uint32) << 16).view(np.float32)
+    mag = np.concatenate([mag, mag])
+    amaxes = []
+    for k in (-40, -20, -10, -4, -1, 0, 1, 4, 12):
+        a = np.array([448.0 * 2.0 ** k], np.float32)
+        a_bits = int(torch.from_numpy(a).to(torch.bfloat16).view(torch.int16).item()) & 0xFFFF
+        amaxes += [a_bits, a_bits + 1, a_bits - 1]                # s a power of two, just above, just below
+    for v in (1.0, 3.0, 0.1, 7.7e-3, 1234.5):
+        amaxes.append(int(torch.tensor([v]).to(torch.bfloat16).view(torch.int16).item()) & 0xFFFF)
+    blocks = []
+    for a_bits in amaxes:
+        a = float(np.array([a_bits << 16], np.uint32).view(np.float32)[0])
+        sel = bits[mag <= a]
+        per = 128 * 128 - 1
+        for i in range(0, sel.size, per):
+            blk = np.zeros(128 * 128, np.uint32)
+            chunk = sel[i:i + per]
+            blk[:chunk.size] = chunk
+            blk[-1] = a_bits                                      # the block's amax
+            blocks.append(blk.reshape(128, 128))
+    x = _bf16_from_bits(np.concatenate(blocks, 0))
+    assert x.shape[0] >= 128 * len(amaxes)
+    run_and_compare(x)
+
+
 def test_quantize_outlier_rows_4096():
     run_and_compare(inputs.dense_4096_outliers().A)
 
