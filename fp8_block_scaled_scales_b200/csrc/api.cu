@@ -96,9 +96,47 @@ dg_status_t current_device(DeviceInfo *info, int *device) {
     return info->ok ? DG_OK : DG_ERR_UNSUPPORTED_DEVICE;
 }
 
+namespace {
+// Encoded tensor maps of recent calls, per host thread.  A map depends only on the
+// address, shape, box and swizzle (no device state), so an entry with the same key
+// is the same map; a decode loop that reuses its buffers skips the encoding.
+struct TmapEntry {
+    const void *base;
+    uint64_t rows, cols;
+    uint32_t box_rows, box_cols;
+    int dtype, elem_bytes, swizzle;
+    CUtensorMap map;
+};
+constexpr int kTmapCache = 32;
+thread_local TmapEntry t_tmaps[kTmapCache];
+thread_local int t_tmap_used = 0, t_tmap_next = 0;
+}  // namespace
+
 dg_status_t make_tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, int elem_bytes,
                          uint64_t rows, uint64_t cols, uint32_t box_rows, uint32_t box_cols,
                          CUtensorMapSwizzle swizzle) {
+    for (int i = 0; i < t_tmap_used; ++i) {
+        const TmapEntry &e = t_tmaps[i];
+        if (e.base == base && e.rows == rows && e.cols == cols && e.box_rows == box_rows &&
+            e.box_cols == box_cols && e.dtype == static_cast<int>(dtype) && e.elem_bytes == elem_bytes &&
+            e.swizzle == static_cast<int>(swizzle)) {
+            *map = e.map;
+            return DG_OK;
+        }
+    }
+    const dg_status_t st = encode_tmap_2d(map, base, dtype, elem_bytes, rows, cols, box_rows, box_cols, swizzle);
+    if (st != DG_OK) return st;
+    TmapEntry &e = t_tmaps[t_tmap_next];
+    e = TmapEntry{base, rows, cols, box_rows, box_cols, static_cast<int>(dtype), elem_bytes,
+                  static_cast<int>(swizzle), *map};
+    t_tmap_next = (t_tmap_next + 1) % kTmapCache;
+    if (t_tmap_used < kTmapCache) ++t_tmap_used;
+    return DG_OK;
+}
+
+dg_status_t encode_tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, int elem_bytes,
+                           uint64_t rows, uint64_t cols, uint32_t box_rows, uint32_t box_cols,
+                           CUtensorMapSwizzle swizzle) {
     const cuuint64_t dims[2] = {cols, rows};
     const cuuint64_t strides[1] = {cols * static_cast<uint64_t>(elem_bytes)};
     const cuuint32_t box[2] = {box_cols, box_rows};

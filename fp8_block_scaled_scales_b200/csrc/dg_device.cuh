@@ -312,9 +312,10 @@ __device__ __forceinline__ void tmem_wait(uint32_t (&r)[64]) {
 __device__ __forceinline__ void tmem_load16_async(uint32_t taddr, uint32_t (&r)[16]) { tmem_load_async(taddr, r); }
 __device__ __forceinline__ void tmem_wait16(uint32_t (&r)[16]) { tmem_wait(r); }
 
-// Columns per TMEM load in the promotion of the tile and pair kernels.
+// Columns per TMEM load in the promotion of the tile and pair kernels (64: measured
+// fastest, and the 128 x 256 tile kernel then needs no register spills).
 #ifndef DG_PROMO_CHUNK
-#define DG_PROMO_CHUNK 16
+#define DG_PROMO_CHUNK 64
 #endif
 constexpr int kPromoChunk = DG_PROMO_CHUNK;
 

@@ -20,10 +20,14 @@ struct DeviceInfo {
 dg_status_t current_device(DeviceInfo *info, int *device);
 
 // Encodes a 2-D tiled tensor map (row-major [rows][cols] of elem_bytes each)
-// with a box of box_cols x box_rows and the given swizzle.
+// with a box of box_cols x box_rows and the given swizzle.  make_tmap_2d serves
+// repeated keys from a small per-thread cache; encode_tmap_2d always encodes.
 dg_status_t make_tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, int elem_bytes,
                          uint64_t rows, uint64_t cols, uint32_t box_rows, uint32_t box_cols,
                          CUtensorMapSwizzle swizzle);
+dg_status_t encode_tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, int elem_bytes,
+                           uint64_t rows, uint64_t cols, uint32_t box_rows, uint32_t box_cols,
+                           CUtensorMapSwizzle swizzle);
 
 // Time limit for every bounded wait inside the kernels, and test-only switches.
 struct KernelControl {

@@ -197,8 +197,12 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 
     if (warp < 4) {
         regs_dealloc<pair_regs_producer<BN>()>();
-        if (warp == 0 && lane == 0) {
-            // ---------------------------------------------- producer (both CTAs)
+        if ((warp == 0 || warp == 3) && lane == 0) {
+            // --------------------------------------------- producers (both CTAs)
+            // Two threads per CTA, one per parity of the iteration (one thread's
+            // issue of a stage takes longer than the K block's MMAs, measured); with
+            // STAGES even each stage belongs to one thread.
+            const int pr = warp == 0 ? 0 : 1;
             const uint32_t full0 = mapa_shared(smem_u32(&full[0]), 0);  // the even CTA's full[0]
             int it = 0;
             bool ok = true;
@@ -207,6 +211,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                 const int a_row = (2 * w.mp + static_cast<int>(rank)) * 128;
                 const int b_row = w.n0 + static_cast<int>(rank) * (w.narrow ? BN / 4 : BN / 2);
                 for (int kb = 0; kb < Kb; ++kb, ++it) {
+                    if ((it & 1) != pr) continue;  // the other producer's stage
                     const int s = it % STAGES;
                     const uint32_t u = static_cast<uint32_t>(it / STAGES);
                     if (!mbar_wait(&empty[s], (u & 1u) ^ 1u, abort_flag, p.timeout_ns)) {

@@ -196,10 +196,16 @@ __global__ void __launch_bounds__(skinny_threads<FUSED>(), 1)
     grid_dep_wait();  // inputs and outputs are touched only from here on
     grid_dep_launch_dependents();
 
-    if (warp == 0 && lane == 0) {
-        // -------------------------------------------------------------- producer
+    if ((warp == 0 || (!FUSED && warp == 3)) && lane == 0) {
+        // ------------------------------------------------------------- producers
+        // Unfused: two threads, one per parity of the K block (one thread's issue of
+        // a stage takes ~600 cycles, measured; the whole K range is issued up front,
+        // so this halves the time to the last copy).  Fused: warp 3 streams the BF16
+        // slabs, and warp 0 issues every weight slab.
+        const int np = FUSED ? 1 : 2;
+        const int pr = warp == 0 ? 0 : 1;
         uint32_t issued = 0, parity_bits = 0;
-        for (int i = 0; i < nkb; ++i) {
+        for (int i = pr; i < nkb; i += np) {
             const int s = i % STAGES;
             const uint32_t u = static_cast<uint32_t>(i / STAGES);
             const int kb = kb0 + i;

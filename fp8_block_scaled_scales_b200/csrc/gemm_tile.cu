@@ -13,15 +13,15 @@
 // epilogue warpgroups with setmaxnreg (128 x 56 + 256 x 224 = 384 x 168, the
 // registers the block is launched with, for 256-column tiles) -- a split above
 // them would make setmaxnreg.inc wait forever; the launcher checks the count):
-//   warp 0      TMA producer: 128-K slabs of A (128 rows) and B (BN rows) into a
-//               STAGES-deep ring of 128-byte-swizzled shared-memory stages
-//               (demingchina.com/news/60142 §3.3 producer/consumer split, §4.2
-//               swizzle, §4.3 multi-stage ring).
+//   warps 0, 3  TMA producers (one thread each, alternate K blocks): 128-K slabs of
+//               A (128 rows) and B (BN rows) into a STAGES-deep ring of
+//               128-byte-swizzled shared-memory stages (demingchina.com/news/60142
+//               §3.3 producer/consumer split, §4.2 swizzle, §4.3 multi-stage ring).
 //   warps 1-2   MMA issuers: one thread each, alternating K blocks; per K block
 //               four tcgen05.mma (K = 32 each) into that K block's TMEM partial
 //               buffer, then a commit to the stage's "empty" barrier (the stage
 //               is free once the MMAs have read it) and one to the buffer's "full".
-//   warp 3      (kMasked) builds the m-block prefix table, then idles.
+//               (kMasked: warp 3 first builds the m-block prefix table.)
 //   warps 4-11  epilogue: per kb, tcgen05.ld the
 //               partial kPromoChunk columns at a time (promote_kblock), release
 //               the TMEM buffer as soon as the last load has landed, and
@@ -314,8 +314,14 @@ __global__ void __launch_bounds__(kTileThreads, 1)
 
     if (warp < 4) {
         regs_dealloc<regs_producer<BN>()>();
-        if (warp == 0 && lane == 0) {
-            // ------------------------------------------------------------ producer
+        if ((warp == 0 || warp == 3) && lane == 0) {
+            // ----------------------------------------------------------- producers
+            // Two threads, one per parity of the iteration: a thread's issue of one
+            // stage (barrier wait, byte count, two tile copies) takes ~600 cycles,
+            // measured, more than the K block's MMAs, and two threads double the
+            // rate.  With STAGES even each stage belongs to one thread, whose parity
+            // waits then stay in order.
+            const int pr = warp == 0 ? 0 : 1;
             uint32_t issued = 0, parity_bits = 0;
             int it = 0;
             bool ok = true;
@@ -326,6 +332,7 @@ __global__ void __launch_bounds__(kTileThreads, 1)
                 const bool narrow = h >= 0;
                 const int b_row = ti.b_row + (narrow ? h * (BN / 2) : 0);
                 for (int kb = 0; kb < Kb; ++kb, ++it) {
+                    if ((it & 1) != pr) continue;  // the other producer's stage
                     const int s = it % STAGES;
                     const uint32_t u = static_cast<uint32_t>(it / STAGES);
                     if (!mbar_wait(&empty[s], (u & 1u) ^ 1u, abort_flag, p.timeout_ns)) {

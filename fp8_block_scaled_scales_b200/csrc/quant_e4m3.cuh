@@ -3,12 +3,10 @@
 // §3.3 FP32 scales).  Bit-exact contract, for every element x of a block:
 //   s = fl32(amax / 448) (1 if amax == 0);  q = E4M3_rn_satfinite(fl32(x / s)).
 //
-// Division: fl32(x/s) is needed only through its E4M3 rounding.  The code forms
-// y = x * r with r = 1/s correctly rounded (__frcp_rn).  Two roundings of relative
-// size <= 2^-24 each put y within 2 FP32 ulps of x/s, and fl32(x/s) is within half
-// an ulp of it; so unless an E4M3 rounding boundary lies within 3 ulps of y, y and
-// fl32(x/s) round to the same E4M3 code.  Near a boundary (see quantize8) or when
-// r is not finite, the IEEE division x / s is used instead.
+// Division: fl32(x/s) is needed only through its E4M3 rounding, so the code is
+// decided from two products that bracket it (quantize8) and the IEEE division
+// x / s is used only when the bracket straddles an E4M3 rounding boundary or when
+// 1/s is not finite.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -46,9 +44,10 @@ __device__ __forceinline__ uint32_t amax_bits_of(uint32_t m2) { return max(m2 & 
 
 // Block scale from the block's BF16 amax bits, with what the conversion needs.
 struct BlockScale {
-    float s;       // fl32(amax / 448), 1 for an all-zero block
-    float2 r2;     // (1/s, 1/s) correctly rounded
-    bool fast_ok;  // 1/s is finite
+    float s;        // fl32(amax / 448), 1 for an all-zero block
+    float2 rlo2;    // 1/s nudged down and up by a relative 2^-21 (see quantize8)
+    float2 rhi2;
+    bool fast_ok;   // 1/s is finite
 };
 
 __device__ __forceinline__ BlockScale block_scale(uint32_t amax_bits) {
@@ -57,54 +56,47 @@ __device__ __forceinline__ BlockScale block_scale(uint32_t amax_bits) {
     b.s = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
     const float r = __frcp_rn(b.s);
     b.fast_ok = isfinite(r);
-    b.r2 = make_float2(r, r);
+    const float rlo = __fmul_rn(r, 1.0f - 0x1p-21f), rhi = __fmul_rn(r, 1.0f + 0x1p-21f);
+    b.rlo2 = make_float2(rlo, rlo);
+    b.rhi2 = make_float2(rhi, rhi);
     return b;
 }
 
 // Eight BF16 (one 16-byte group) -> eight E4M3 codes.
 //
-// y = x * r is within 3 FP32 ulps of fl32(x / s), so the two round to the same E4M3
-// code unless an E4M3 rounding boundary lies within 3 ulps of y.  Two screens find
-// every such y, branch-free, over the eight values:
-//   - normal range (|y| >= 2^-6): the boundaries are the FP32 values whose mantissa
-//     is ...1000...0 below the three kept bits, i.e. bits[19:0] == 0x80000; y is
-//     within 6 ulps of one iff (bits + 0x80006) & 0xFFFFF <= 12;
-//   - below 2^-6 (E4M3 subnormals, quantum 2^-9): the boundaries are the odd
-//     multiples of 2^-10, i.e. 1024 y an odd integer.  With M = 1.5 * 2^23,
-//     rr = fl32(1024 y + M) holds the nearest integer n to 1024 y in its last bits
-//     (its lowest bit is n's parity), and d = 1024 y - n is exact; 3 ulps of y
-//     below 2^-6 are at most 3 * 2^-20 in these units, so the test is |d| <= 2^-18
-//     with n odd.  Values that are exact E4M3 numbers (n even), zero included, never
-//     fire.
-// Only when a screen fires -- about once in 10^5 values -- are the eight quotients
-// recomputed with IEEE division.  (A screen that sent every |y| < 2^-6 to the
-// division fired in most warps: measured, half the quantizer's time.)
+// The code wanted is E4M3(t), t = fl32(x / s).  With rlo, rhi = 1/s (correctly
+// rounded) times 1 -+ 2^-21 (rounded), ylo = fl32(x rlo) and yhi = fl32(x rhi)
+// bracket t strictly: three roundings of relative size at most 2^-24 each put
+// |ylo| below |x/s| (1 - 2^-21)(1 + 2^-24)^3 < |x/s| (1 - 2^-24) <= |t|, and |yhi|
+// above |t| likewise (FP32 underflow aside, where every candidate is far below the
+// E4M3 range and gets the code of zero).  Rounding to E4M3 is monotone, so when
+// ylo and yhi get the same code, t gets it too.  They differ only when a rounding
+// boundary falls inside the bracket -- for data with an arbitrary amax about once
+// in 10^5 values; more often when x / s lands exactly on a boundary, as it can when
+// s is a power of two -- and then the eight quotients are recomputed with IEEE
+// division.  Per value this costs two multiplies and two conversions, no bit tests.
+// (Checked exhaustively on the CPU for every BF16 x and every block amax.)
 __device__ __forceinline__ uint2 quantize8(uint4 v, const BlockScale &b) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    const float2 k1024 = make_float2(1024.0f, 1024.0f);
-    const float2 magic = make_float2(0x1.8p23f, 0x1.8p23f);
-    const float2 neg_magic = make_float2(-0x1.8p23f, -0x1.8p23f);
-    float2 x[4], y[4];
-    uint32_t dmin = 0xFFFFFFFFu, sub = 0;
+    float2 x[4], lo[4], hi[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         x[j] = make_float2(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xFFFF0000u));
-        y[j] = __fmul2_rn(x[j], b.r2);
-        dmin = min(dmin, (__float_as_uint(y[j].x) + 0x80006u) & 0xFFFFFu);
-        dmin = min(dmin, (__float_as_uint(y[j].y) + 0x80006u) & 0xFFFFFu);
-        const float2 rr = __ffma2_rn(y[j], k1024, magic);
-        const float2 n = __fadd2_rn(rr, neg_magic);
-        const float2 d = __ffma2_rn(y[j], k1024, make_float2(-n.x, -n.y));
-        sub |= (fabsf(d.x) <= 0x1p-18f) ? (__float_as_uint(rr.x) & 1u) : 0u;
-        sub |= (fabsf(d.y) <= 0x1p-18f) ? (__float_as_uint(rr.y) & 1u) : 0u;
-    }
-    if (__builtin_expect(dmin <= 12u || sub != 0u || !b.fast_ok, 0)) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) y[j] = make_float2(__fdiv_rn(x[j].x, b.s), __fdiv_rn(x[j].y, b.s));
+        lo[j] = __fmul2_rn(x[j], b.rlo2);
+        hi[j] = __fmul2_rn(x[j], b.rhi2);
     }
     uint2 out;
-    out.x = e4m3x4(y[0].x, y[0].y, y[1].x, y[1].y);
-    out.y = e4m3x4(y[2].x, y[2].y, y[3].x, y[3].y);
+    out.x = e4m3x4(hi[0].x, hi[0].y, hi[1].x, hi[1].y);
+    out.y = e4m3x4(hi[2].x, hi[2].y, hi[3].x, hi[3].y);
+    const uint32_t lx = e4m3x4(lo[0].x, lo[0].y, lo[1].x, lo[1].y);
+    const uint32_t ly = e4m3x4(lo[2].x, lo[2].y, lo[3].x, lo[3].y);
+    if (__builtin_expect(((out.x ^ lx) | (out.y ^ ly)) != 0u || !b.fast_ok, 0)) {
+        float2 y[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) y[j] = make_float2(__fdiv_rn(x[j].x, b.s), __fdiv_rn(x[j].y, b.s));
+        out.x = e4m3x4(y[0].x, y[0].y, y[1].x, y[1].y);
+        out.y = e4m3x4(y[2].x, y[2].y, y[3].x, y[3].y);
+    }
     return out;
 }
 
