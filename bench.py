@@ -70,6 +70,19 @@ SKINNY_GRAPH_STEPS = 240
 # keyed by workload, kernel file and the hash of that file's code; a kernel changed
 # since the capture reports null.
 NCU_TRAFFIC = {
+    # tile_gemm_kernel<256,kDense,4,2,0>, dense 4096^3 (1% outlier rows): 33.60 MB read + 2.14 MB written
+    ("dense_4096_outliers", "gemm_tile.cu", "d24505a938289113"): 35738368,
+    # tile_gemm_kernel<256,kDense,4,2,0>, dense 8192^3: 435.58 MB read + 120.47 MB written
+    ("dense_8192", "gemm_tile.cu", "d24505a938289113"): 556048384,
+    # tile_gemm_kernel<256,kContiguous,4,2,0>, 8 experts N=K=4096: 210.29 MB read + 116.65 MB written
+    ("moe_g8", "gemm_tile.cu", "d24505a938289113"): 326939904,
+    # tile_gemm_kernel<256,kContiguous,4,2,0>, 64 experts N=2048 K=7168: 1410.22 MB read + 145.02 MB written
+    ("moe_g64_zipf", "gemm_tile.cu", "d24505a938289113"): 1555234048,
+    # skinny_gemm_kernel<16,8,8,0> M=16; <64,8,8,0> M=64; <128,6,4,0> M=128; fused <16,8,8,1> M=1 (N=K=4096)
+    ("skinny_m16", "gemm_skinny.cu", "fc4008f58dc9f455"): 16875008,
+    ("skinny_m64", "gemm_skinny.cu", "fc4008f58dc9f455"): 17073408,
+    ("skinny_m128", "gemm_skinny.cu", "fc4008f58dc9f455"): 17336576,
+    ("skinny_m1", "gemm_skinny.cu", "fc4008f58dc9f455"): 16833024,
 }
 
 KERNEL_HEADERS = ("dg_device.cuh", "quant_e4m3.cuh", "dg_internal.h")  # device code the kernels include
