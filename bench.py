@@ -577,6 +577,32 @@ def e2e_ms(plans, steps, stream):
     return e0.elapsed_time(e1) / steps, mode, h2d, d2h
 
 
+def c_abi_enqueue_us(p, calls=200):
+    """Host time per step of the library's own C calls (ctypes, arguments prepared),
+    the launches queued behind a GPU sleep so that no call waits for the device."""
+    import ctypes
+    L = p.b.lib()
+    st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    ptr = lambda t: ctypes.c_void_p(t.data_ptr())
+    w = p.w
+    if p.fused:
+        steps = [(L.dg_fp8_gemm_blockscaled_bf16a,
+                  (ptr(p.A), ptr(p.qb), ptr(p.sb), ptr(p.C), ptr(p.qa), ptr(p.sa), w.M, w.N, w.K, st))]
+    else:
+        steps = [(L.dg_quantize_blockwise, (ptr(p.A), w.M, w.K, ptr(p.qa), ptr(p.sa), st)),
+                 (L.dg_fp8_gemm_blockscaled, (ptr(p.qa), ptr(p.sa), ptr(p.qb), ptr(p.sb), ptr(p.C), w.M, w.N, w.K, st))]
+    torch.cuda.synchronize()
+    torch.cuda._sleep(int(1.5e9 * 0.01))
+    t0 = time.perf_counter()
+    for _ in range(calls):
+        for f, a in steps:
+            if f(*a) != 0:
+                raise SystemExit("C call failed")
+    dt = time.perf_counter() - t0
+    torch.cuda.synchronize()
+    return dt / calls * 1e6
+
+
 def roofline_entry(bound, achieved, peaks, traffic, algorithmic_bytes, kernel, kernel_ms):
     if bound == "hbm":
         peak, spec, unit = peaks["hbm_gbs"], SPEC_HBM_GBS, "GB/s"
@@ -632,6 +658,7 @@ def measure(name, plans, args, world, flush, stream, peaks, cpu_ws=None, cpu_gfl
         entry["cold_step_ms"] = round(max_over_ranks(statistics.median([c[0] for c in cold]), world), 5)
         entry["cold_value"] = round(aggregate_rate(world, p.step_bytes, entry["cold_step_ms"]) / 1e9, 1)
         entry["step_bytes"] = int(p.step_bytes)
+        entry["c_abi_enqueue_us_per_step"] = round(c_abi_enqueue_us(p), 2)
         launches = p.launches
     else:
         whole = [lambda: [pl.step() for pl in plans]]
@@ -719,7 +746,7 @@ def run_dg(args):
            "host_enqueue_us_per_step": e["host_enqueue_us_per_step"]}
     if "cpu_baseline" in e:
         out["cpu_baseline"] = e["cpu_baseline"]
-    for k in ("kernels_ms", "gemm_tflops", "timing"):
+    for k in ("kernels_ms", "gemm_tflops", "timing", "cold_step_ms", "cold_value", "c_abi_enqueue_us_per_step"):
         if k in e:
             out[k] = e[k]
     cs = clocks.summary()
