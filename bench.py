@@ -56,7 +56,6 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-FUSED_MAX_M = 1  # the library quantizes A inside the skinny GEMM up to this M
 E2E_PIPELINE_MIN_BYTES = 4 << 20  # host<->device bytes per step above which e2e overlaps copies
 L2_FLUSH_BYTES = 256 << 20
 L2_BYTES = 126 << 20
@@ -70,19 +69,6 @@ SKINNY_GRAPH_STEPS = 240
 # keyed by workload, kernel file and the hash of that file's code; a kernel changed
 # since the capture reports null.
 NCU_TRAFFIC = {
-    # tile_gemm_kernel<256,kDense,4,2,0>, dense 4096^3 (1% outlier rows): 33.60 MB read + 2.14 MB written
-    ("dense_4096_outliers", "gemm_tile.cu", "d24505a938289113"): 35738368,
-    # tile_gemm_kernel<256,kDense,4,2,0>, dense 8192^3: 435.58 MB read + 120.47 MB written
-    ("dense_8192", "gemm_tile.cu", "d24505a938289113"): 556048384,
-    # tile_gemm_kernel<256,kContiguous,4,2,0>, 8 experts N=K=4096: 210.29 MB read + 116.65 MB written
-    ("moe_g8", "gemm_tile.cu", "d24505a938289113"): 326939904,
-    # tile_gemm_kernel<256,kContiguous,4,2,0>, 64 experts N=2048 K=7168: 1410.22 MB read + 145.02 MB written
-    ("moe_g64_zipf", "gemm_tile.cu", "d24505a938289113"): 1555234048,
-    # skinny_gemm_kernel<16,8,8,0> M=16; <64,8,8,0> M=64; <128,6,4,0> M=128; fused <16,8,8,1> M=1 (N=K=4096)
-    ("skinny_m16", "gemm_skinny.cu", "fc4008f58dc9f455"): 16875008,
-    ("skinny_m64", "gemm_skinny.cu", "fc4008f58dc9f455"): 17073408,
-    ("skinny_m128", "gemm_skinny.cu", "fc4008f58dc9f455"): 17336576,
-    ("skinny_m1", "gemm_skinny.cu", "fc4008f58dc9f455"): 16833024,
 }
 
 KERNEL_HEADERS = ("dg_device.cuh", "quant_e4m3.cuh", "dg_internal.h")  # device code the kernels include
@@ -121,7 +107,7 @@ def load_peaks():
 
 # ------------------------------------------------------------------ workloads
 WORKLOADS = ("dense_4096_outliers", "dense_512", "dense_8192", "skinny_m1", "skinny_m16", "skinny_m64",
-             "skinny_m128", "moe_g8", "moe_g64_zipf", "moe_masked_g8", "dense_4096_outliers_1x128",
+             "skinny_m128", "skinny_m1_fused", "skinny_m16_fused", "moe_g8", "moe_g64_zipf", "moe_masked_g8", "dense_4096_outliers_1x128",
              "moe_g64_zipf+dense_8192")
 # the default run: every benchmark workload, the last one on the top level
 SUITE = ("dense_512", "dense_4096_outliers", "skinny_m1", "skinny_m16", "skinny_m64", "skinny_m128", "moe_g8",
@@ -134,6 +120,8 @@ def make_workload(name):
     from fp8_block_scaled_scales_b200 import inputs
     if name.endswith("_1x128"):  # the same data, per-token activation scales
         name = name[:-len("_1x128")]
+    if name.endswith("_fused"):  # the same data, A quantized inside the skinny GEMM (one launch)
+        name = name[:-len("_fused")]
     if name == "dense_4096_outliers":
         return inputs.dense_4096_outliers()
     if name == "dense_512":
@@ -399,7 +387,7 @@ class Plan:
         if self.rowscale:
             self.cfg = dict(self.cfg, workload=name, a_scales="one per row and 128-K group (K-block-major)")
         self.skinny = not (self.grouped or self.masked or self.rowscale) and w.M <= 128
-        self.fused = self.skinny and w.M <= FUSED_MAX_M
+        self.fused = self.skinny and name.endswith("_fused")
         self.kernel_file = ("gemm_tile.cu" if (self.grouped or self.masked)
                             else "gemm_skinny.cu" if self.skinny else "gemm_pair.cu")
         self.A_host = w.A.contiguous().reshape(rows_a, w.K)  # masked: the [G][M_max] slabs as rows
@@ -450,7 +438,8 @@ class Plan:
         x = self.A if x is None else x
         if self.fused:
             self.b.gemm_blockscaled_bf16a(x, self.qb if qb is None else qb, self.sb if sb is None else sb,
-                                          C=self.C if Cout is None else Cout, QA=self.qa, sA=self.sa)
+                                          C=self.C if Cout is None else Cout, QA=self.qa, sA=self.sa,
+                                          kernel="fused")
         else:
             self.quantize(x)
             self.gemm(Cout, qb, sb)
@@ -586,8 +575,8 @@ def c_abi_enqueue_us(p, calls=200):
     ptr = lambda t: ctypes.c_void_p(t.data_ptr())
     w = p.w
     if p.fused:
-        steps = [(L.dg_fp8_gemm_blockscaled_bf16a,
-                  (ptr(p.A), ptr(p.qb), ptr(p.sb), ptr(p.C), ptr(p.qa), ptr(p.sa), w.M, w.N, w.K, st))]
+        steps = [(L.dg_fp8_gemm_blockscaled_bf16a_select,
+                  (ptr(p.A), ptr(p.qb), ptr(p.sb), ptr(p.C), ptr(p.qa), ptr(p.sa), w.M, w.N, w.K, 4, st))]
     else:
         steps = [(L.dg_quantize_blockwise, (ptr(p.A), w.M, w.K, ptr(p.qa), ptr(p.sa), st)),
                  (L.dg_fp8_gemm_blockscaled, (ptr(p.qa), ptr(p.sa), ptr(p.qb), ptr(p.sb), ptr(p.C), w.M, w.N, w.K, st))]
@@ -773,7 +762,7 @@ def run_reference(args):
     cfg = facts[0][3] if len(ws) == 1 else {"workload": name, "parts": [f[3] for f in facts]}
     skinny = len(ws) == 1 and not hasattr(ws[0], "counts") and ws[0].M <= 128
     unit = "GB/s" if skinny else "TFLOP/s"
-    bpf = skinny_step_bytes(ws[0].M, ws[0].N, ws[0].K, ws[0].M <= FUSED_MAX_M) / facts[0][0] if skinny else 0.0
+    bpf = skinny_step_bytes(ws[0].M, ws[0].N, ws[0].K, name.endswith("_fused")) / facts[0][0] if skinny else 0.0
     gflop = args.oracle_gflop / 4
     times = []
     for i in range(args.warmup + args.steps):

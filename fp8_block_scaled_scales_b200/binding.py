@@ -20,10 +20,11 @@ DG_OK = 0
 STATUS_NAMES = {0: "DG_OK", 1: "DG_ERR_INVALID_ARG", 2: "DG_ERR_SHAPE", 3: "DG_ERR_ALIGNMENT",
                 4: "DG_ERR_UNSUPPORTED_DEVICE", 5: "DG_ERR_CUDA", 6: "DG_ERR_TIMEOUT",
                 7: "DG_ERR_GROUP_OFFSETS"}
-KERNELS = {"auto": 0, "tile": 1, "skinny": 2, "pair": 3}
+KERNELS = {"auto": 0, "tile": 1, "skinny": 2, "pair": 3, "fused": 4}
 
 # every symbol include/dg.h declares
 EXPORTS = ("dg_quantize_blockwise", "dg_fp8_gemm_blockscaled", "dg_fp8_gemm_blockscaled_bf16a",
+           "dg_fp8_gemm_blockscaled_bf16a_select",
            "dg_fp8_grouped_gemm_contiguous", "dg_fp8_grouped_gemm_masked", "dg_quantize_1x128",
            "dg_fp8_gemm_1x128", "dg_fp8_gemm_1x128_select",
            "dg_fp8_gemm_blockscaled_select", "dg_status_string", "dg_get_last_device_status",
@@ -53,13 +54,14 @@ def lib() -> ctypes.CDLL:
     L.dg_fp8_gemm_blockscaled.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp]
     L.dg_fp8_gemm_blockscaled_select.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, vp]
     L.dg_fp8_gemm_blockscaled_bf16a.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp]
+    L.dg_fp8_gemm_blockscaled_bf16a_select.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, vp]
     L.dg_fp8_grouped_gemm_contiguous.argtypes = [vp, vp, vp, vp, vp, vp, i64, i32, i64, i64, vp]
     L.dg_fp8_grouped_gemm_masked.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, i64, i64, vp]
     L.dg_quantize_1x128.argtypes = [vp, i64, i64, vp, vp, vp]
     L.dg_fp8_gemm_1x128.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp]
     L.dg_fp8_gemm_1x128_select.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, vp]
     for f in ("dg_quantize_blockwise", "dg_fp8_gemm_blockscaled", "dg_fp8_gemm_blockscaled_select",
-              "dg_fp8_gemm_blockscaled_bf16a",
+              "dg_fp8_gemm_blockscaled_bf16a", "dg_fp8_gemm_blockscaled_bf16a_select",
               "dg_fp8_grouped_gemm_contiguous", "dg_fp8_grouped_gemm_masked", "dg_get_last_device_status",
               "dg_quantize_1x128", "dg_fp8_gemm_1x128", "dg_fp8_gemm_1x128_select"):
         getattr(L, f).restype = ctypes.c_int
@@ -127,10 +129,11 @@ def gemm_blockscaled(A, sA, B, sB, C=None, kernel: str = "auto", stream=None):
     return C
 
 
-def gemm_blockscaled_bf16a(A, B, sB, C=None, QA=None, sA=None, stream=None):
+def gemm_blockscaled_bf16a(A, B, sB, C=None, QA=None, sA=None, kernel: str = "auto", stream=None):
     """C[M][N] (bf16) = quantize(A)[M][K] . B[N][K]^T from BF16 activations A.
 
-    Returns (C, QA, sA): A's E4M3 codes and 128x128 block scales are outputs too."""
+    Returns (C, QA, sA): A's E4M3 codes and 128x128 block scales are outputs too.
+    kernel="fused" (M <= 16) quantizes A inside the skinny GEMM, in one launch."""
     M, K = A.shape
     B = _u8(B)
     N = B.shape[0]
@@ -141,8 +144,8 @@ def gemm_blockscaled_bf16a(A, B, sB, C=None, QA=None, sA=None, stream=None):
         QA = torch.empty((M, K), dtype=torch.uint8, device=dev)
     if sA is None:
         sA = torch.empty(((M + 127) // 128, (K + 127) // 128), dtype=torch.float32, device=dev)
-    _check(lib().dg_fp8_gemm_blockscaled_bf16a(_p(A), _p(B), _p(sB), _p(C), _p(_u8(QA)), _p(sA), M, N, K,
-                                               _stream(stream)),
+    _check(lib().dg_fp8_gemm_blockscaled_bf16a_select(_p(A), _p(B), _p(sB), _p(C), _p(_u8(QA)), _p(sA), M, N, K,
+                                                      KERNELS[kernel], _stream(stream)),
            "dg_fp8_gemm_blockscaled_bf16a")
     return C, QA, sA
 

@@ -153,7 +153,7 @@ using namespace dg;
 
 extern "C" {
 
-int dg_version(void) { return 102; }
+int dg_version(void) { return 103; }
 
 const char *dg_status_string(dg_status_t s) {
     switch (s) {
@@ -275,11 +275,16 @@ dg_status_t dg_fp8_gemm_1x128(const uint8_t *A, const float *sA_t, const uint8_t
     return dg_fp8_gemm_1x128_select(A, sA_t, B, sB, C_bf16, M, N, K, DG_KERNEL_AUTO, stream);
 }
 
-dg_status_t dg_fp8_gemm_blockscaled_bf16a(const void *A_bf16, const uint8_t *B, const float *sB, void *C_bf16,
-                                          uint8_t *QA, float *sA, int64_t M, int64_t N, int64_t K,
-                                          cudaStream_t stream) {
+dg_status_t dg_fp8_gemm_blockscaled_bf16a_select(const void *A_bf16, const uint8_t *B, const float *sB,
+                                                 void *C_bf16, uint8_t *QA, float *sA, int64_t M, int64_t N,
+                                                 int64_t K, dg_kernel_t kernel, cudaStream_t stream) {
     if (M < 0 || N < 0 || K <= 0 || K % 16 != 0 || N % 16 != 0) return DG_ERR_SHAPE;
     if (M > 0x7FFFFFFFLL || N > 0x7FFFFFFFLL || K > 0x7FFFFFFFLL) return DG_ERR_SHAPE;
+    if (kernel != DG_KERNEL_AUTO && kernel != DG_KERNEL_TILE && kernel != DG_KERNEL_SKINNY &&
+        kernel != DG_KERNEL_PAIR && kernel != DG_KERNEL_SKINNY_FUSED)
+        return DG_ERR_INVALID_ARG;
+    if ((kernel == DG_KERNEL_SKINNY && M > 128) || (kernel == DG_KERNEL_SKINNY_FUSED && M > kFusedMaxM))
+        return DG_ERR_SHAPE;
     if (M == 0 || N == 0) return DG_OK;
     if (!A_bf16) return DG_ERR_INVALID_ARG;
     dg_status_t st = check_gemm_common(QA, sA, B, sB, C_bf16);
@@ -288,14 +293,20 @@ dg_status_t dg_fp8_gemm_blockscaled_bf16a(const void *A_bf16, const uint8_t *B, 
     DeviceInfo dev;
     st = current_device(&dev, nullptr);
     if (st != DG_OK) return st;
-    if (M <= kFusedMaxM) {
+    if (kernel == DG_KERNEL_SKINNY_FUSED) {
         // one launch: the skinny kernel quantizes A itself and writes QA, sA on the way
         GemmArgs a = {QA, sA, B, sB, C_bf16, nullptr, M, N, K, 0};
         return launch_skinny_gemm_fused(a, A_bf16, QA, sA, dev, stream);
     }
     st = launch_quantize(A_bf16, M, K, QA, sA, dev, stream);
     if (st != DG_OK) return st;
-    return dg_fp8_gemm_blockscaled_select(QA, sA, B, sB, C_bf16, M, N, K, DG_KERNEL_AUTO, stream);
+    return dg_fp8_gemm_blockscaled_select(QA, sA, B, sB, C_bf16, M, N, K, kernel, stream);
+}
+
+dg_status_t dg_fp8_gemm_blockscaled_bf16a(const void *A_bf16, const uint8_t *B, const float *sB, void *C_bf16,
+                                          uint8_t *QA, float *sA, int64_t M, int64_t N, int64_t K,
+                                          cudaStream_t stream) {
+    return dg_fp8_gemm_blockscaled_bf16a_select(A_bf16, B, sB, C_bf16, QA, sA, M, N, K, DG_KERNEL_AUTO, stream);
 }
 
 dg_status_t dg_fp8_grouped_gemm_masked(const uint8_t *A, const float *sA, const uint8_t *B, const float *sB,

@@ -82,10 +82,11 @@ dg_status_t launch_pair_gemm(const GemmArgs &a, const DeviceInfo &dev, cudaStrea
 dg_status_t launch_pair_gemm_n128(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream);
 dg_status_t launch_skinny_gemm(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream);
 // M <= kFusedMaxM with BF16 A quantized inside the GEMM; a.A and a.sA are unused.
-// Measured (N = K = 4096, cold L2): one launch beats quantizer + GEMM at M = 1
-// (16.4 vs 17.4 us) and loses from M = 2 on (18.4 vs 17.4 us), where the per-K-block
-// quantization chain, repeated by every N block's CTAs, outgrows the launch it saves.
-constexpr int64_t kFusedMaxM = 1;
+// Chosen explicitly (DG_KERNEL_SKINNY_FUSED): in a graph of back-to-back steps
+// (N = K = 4096) the quantizer + GEMM pair, whose GEMM starts its weight prefetch
+// while the quantizer runs, is as fast or faster (6.65 vs 6.9-7.0 us at M = 1-2;
+// 7.1 vs 10.3 us at M = 16), so the automatic dispatch never picks it.
+constexpr int64_t kFusedMaxM = 16;
 dg_status_t launch_skinny_gemm_fused(const GemmArgs &a, const void *A_bf16, uint8_t *qa_out, float *sa_out,
                                      const DeviceInfo &dev, cudaStream_t stream);
 // one scale per row and 128-column group, written K-block-major: St[ceil(cols/128)][rows]

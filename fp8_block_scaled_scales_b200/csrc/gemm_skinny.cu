@@ -16,18 +16,19 @@
 // memory and writes them as BF16.  The order is fixed, so the result is
 // deterministic (no float atomics; demingchina.com/news/60142 §6.4).
 //
-// Fused activation quantization (FUSED): A arrives as BF16 (TMA brings each K
-// block's M x 128 slab into a ring) and four more warps quantize it per 128x128
-// block (for M <= 128 the block of K block kb is rows 0..M-1 x its 128 columns)
-// straight into the MMA's shared-memory stage, in the
+// Fused activation quantization (FUSED): A arrives as BF16 and four more warps
+// quantize it per 128x128 block (for M <= 16 the block of K block kb is rows
+// 0..M-1 x its 128 columns) straight into the MMA's shared-memory stage, in the
 // 128-byte-swizzled K-major layout TMA would have written, with exactly the
 // arithmetic of the block quantizer (quant_e4m3.cuh).  The step before the GEMM
 // thus needs no launch of its own (2kiu.com/news/5461879 §5: activation scales
-// are recomputed on every call).  The CTAs of the first N block also write the
-// codes and scales out, so the caller gets the same Q, S as from the quantizer.
-// Every N block's CTAs repeat the quantization of their K range, and each K
-// block's conversion sits on its MMA's critical path, so the one launch pays
-// only for a single token row; the library uses it for M = 1.
+// are recomputed on every call).  Each warp owns every fourth K block: it loads
+// the block's M x 128 values from global memory, reduces amax with shuffles and
+// converts, so four K blocks are quantized at once and no block waits on a
+// CTA-wide barrier; the weight stream does not wait for the quantizer.  The CTAs
+// of the first N block also write the codes and scales out, so the caller gets
+// the same Q, S as from the quantizer.  Every N block's CTAs repeat the
+// quantization of their K range (M x K values, small next to the weights).
 #include <cuda_bf16.h>
 
 #include "dg_device.cuh"
@@ -46,7 +47,7 @@ struct SkinnyParams {
     int *status;  // device status word
     int debug_flags;  // bit 0 (tests): the producer never fills stage 0, so a wait must time out
     // FUSED only: BF16 A [M][K], and the codes / scales written by the first N block
-    const uint16_t *Xa;
+    const uint4 *Xa;
     int K;
     uint8_t *qa_out;
     float *sa_out;
@@ -95,23 +96,20 @@ __device__ __forceinline__ void tmem_load16(uint32_t taddr, float (&v)[16]) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-template <int MP, int STAGES, int NBUF, int RA>
+template <int MP, int STAGES, int NBUF>
 struct SkinnySmem {
     static constexpr uint32_t kWBytes = 128 * 128;  // weight slab: 128 rows of B x 128 K
     static constexpr uint32_t kXBytes = MP * 128;   // token slab: MP rows of A x 128 K
-    static constexpr uint32_t kABytes = MP * 256;   // FUSED: BF16 token slab, MP rows x 128 K, unswizzled
     static constexpr uint32_t kOffW = 0;
     static constexpr uint32_t kOffX = kOffW + STAGES * kWBytes;
-    static constexpr uint32_t kOffA = kOffX + STAGES * kXBytes;  // FUSED: ring of RA BF16 slabs
-    static constexpr uint32_t kStageEnd = kOffA + RA * kABytes;
+    static constexpr uint32_t kStageEnd = kOffX + STAGES * kXBytes;
     static constexpr uint32_t kRedBytes = MP * 128 * 4;  // FP32 partial, [MP][128]
     static constexpr uint32_t kDataBytes = kStageEnd > kRedBytes ? kStageEnd : kRedBytes;
     static constexpr uint32_t kOffBar = kDataBytes;
-    static constexpr uint32_t kOffMisc = kOffBar + 8 * (2 * STAGES + 2 * NBUF + 2 + 2 * RA);
-    // misc: TMEM address (0), abort flag (4), FUSED quantizer's stage flag (8)
-    static constexpr uint32_t kOffScaleA = kOffMisc + 16;          // FUSED: A scale of each stage
-    static constexpr uint32_t kOffQRed = kOffScaleA + 4 * STAGES;  // FUSED: amax partials, 2 x 4
-    static constexpr uint32_t kBytes = kOffQRed + 32;
+    static constexpr uint32_t kOffMisc = kOffBar + 8 * (2 * STAGES + 2 * NBUF + 2);
+    // misc: TMEM address (0), abort flag (4)
+    static constexpr uint32_t kOffScaleA = kOffMisc + 16;  // FUSED: A scale of each stage
+    static constexpr uint32_t kBytes = kOffScaleA + 4 * STAGES;
     static constexpr uint32_t kDynamicBytes = kBytes + 1024;
 };
 
@@ -126,9 +124,7 @@ __global__ void __launch_bounds__(skinny_threads<FUSED>(), 1)
     skinny_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                        const SkinnyParams p) {
     constexpr int kThreads = skinny_threads<FUSED>();
-    constexpr int RA = 4;                  // FUSED: BF16 slabs in flight ahead of the quantizer
-    constexpr int kRing = FUSED ? RA : 0;  // ring slots laid out in shared memory
-    using L = SkinnySmem<MP, STAGES, NBUF, kRing>;
+    using L = SkinnySmem<MP, STAGES, NBUF>;
     static_assert(STAGES % 2 == 0 && NBUF % 2 == 0, "each MMA thread must own its stages and buffers");
     constexpr uint32_t kTmemCols = tmem_cols_for(NBUF * MP);
     constexpr uint32_t kIdesc = idesc_e4m3_f32(128, MP);
@@ -140,13 +136,10 @@ __global__ void __launch_bounds__(skinny_threads<FUSED>(), 1)
     uint64_t *tfull = empty + STAGES;
     uint64_t *tempty = tfull + NBUF;
     uint64_t *mdone = tempty + NBUF;
-    uint64_t *afull = mdone + 2;       // FUSED: BF16 slab landed
-    uint64_t *aempty = afull + kRing;  // FUSED: BF16 slab converted
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
     float *red = reinterpret_cast<float *>(smem);  // reuses the stage memory after the K loop
     float *sa_stage = reinterpret_cast<float *>(smem + L::kOffScaleA);
-    uint32_t *qred = reinterpret_cast<uint32_t *>(smem + L::kOffQRed);
 
     const int warp = static_cast<int>(threadIdx.x >> 5);
     const int lane = lane_id();
@@ -176,14 +169,10 @@ __global__ void __launch_bounds__(skinny_threads<FUSED>(), 1)
             mbar_init(&tempty[b], 4);
         }
         for (int q = 0; q < 2; ++q) mbar_init(&mdone[q], 1);
-        for (int r = 0; r < kRing; ++r) {
-            mbar_init(&afull[r], 1);
-            mbar_init(&aempty[r], 1);
-        }
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmW);
-        tma_prefetch_desc(&tmX);
+        if (!FUSED) tma_prefetch_desc(&tmX);
     }
     if (warp == 3) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -196,13 +185,12 @@ __global__ void __launch_bounds__(skinny_threads<FUSED>(), 1)
     grid_dep_wait();  // inputs and outputs are touched only from here on
     grid_dep_launch_dependents();
 
-    if ((warp == 0 || (!FUSED && warp == 3)) && lane == 0) {
+    if ((warp == 0 || warp == 3) && lane == 0) {
         // ------------------------------------------------------------- producers
-        // Unfused: two threads, one per parity of the K block (one thread's issue of
-        // a stage takes ~600 cycles, measured; the whole K range is issued up front,
-        // so this halves the time to the last copy).  Fused: warp 3 streams the BF16
-        // slabs, and warp 0 issues every weight slab.
-        const int np = FUSED ? 1 : 2;
+        // Two threads, one per parity of the K block (one thread's issue of a stage
+        // takes ~600 cycles, measured; the whole K range is issued up front, so this
+        // halves the time to the last copy).
+        const int np = 2;
         const int pr = warp == 0 ? 0 : 1;
         uint32_t issued = 0, parity_bits = 0;
         for (int i = pr; i < nkb; i += np) {
@@ -226,29 +214,6 @@ __global__ void __launch_bounds__(skinny_threads<FUSED>(), 1)
             if (issued & (1u << s))
                 if (!mbar_wait(&full[s], (parity_bits >> s) & 1u, &never, p.timeout_ns))
                     record_failure(p.status, kStatusTimeout, 10, -1 - s);
-    } else if (FUSED && warp == 3 && lane == 0) {
-        // ------------------------------------ BF16 slab producer (FUSED)
-        // Its own thread, so that the weight stream never waits for the quantizer:
-        // slab i goes to ring slot i % RA, RA slabs ahead of the quantizer.
-        int a_issued = 0;
-        for (int i = 0; i < nkb; ++i) {
-            const int ra = i % RA;
-            const uint32_t ua = static_cast<uint32_t>(i / RA);
-            if (!mbar_wait(&aempty[ra], (ua & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
-                record_failure(p.status, kStatusTimeout, 14, i);
-                *abort_flag = 1;
-                break;
-            }
-            mbar_arrive_expect_tx(&afull[ra], L::kABytes);
-            tma_load_2d(smem + L::kOffA + ra * L::kABytes, &tmX, &afull[ra], (kb0 + i) * 128, 0);
-            a_issued = i + 1;
-        }
-        const int never = 0;
-        for (int r = 0; r < RA && r < a_issued; ++r) {  // the last slab of each ring slot
-            const int last = r + ((a_issued - 1 - r) / RA) * RA;
-            if (!mbar_wait(&afull[r], static_cast<uint32_t>(last / RA) & 1u, &never, p.timeout_ns))
-                record_failure(p.status, kStatusTimeout, 14, -1 - r);
-        }
     } else if ((warp == 1 || warp == 2) && lane == 0) {
         // -------------------------------------------------- MMA (two threads)
         // Thread q issues K blocks i with i % 2 == q; with STAGES and NBUF even
@@ -287,80 +252,80 @@ __global__ void __launch_bounds__(skinny_threads<FUSED>(), 1)
         }
     } else if (FUSED && warp >= 8) {
         // ------------------------------------------ activation quantizer (FUSED)
-        // Per K block, all 128 threads: read the BF16 slab from its ring slot
-        // (MP/16 items of one row x 16 columns per thread), reduce amax over the
-        // block, and write the codes into the stage in the swizzled K-major layout
-        // TMA would produce: row r's 16-byte group j at byte r*128 + ((j ^ (r % 8)) * 16).
-        const int qt = static_cast<int>(threadIdx.x) - 256;
-        const int qw = qt >> 5;
-        constexpr int kItems = MP / 16;
-        volatile int *stage_ok = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 8);
-        for (int i = 0; i < nkb; ++i) {
+        // Warp qw quantizes K blocks qw, qw + 4, ...: item (row r, 8-column group g)
+        // = lane + 32 t holds A[r][kb*128 + 8g .. +7]; rows past M and columns past K
+        // are zero and quantize to +0.  The codes go where TMA would have put them in
+        // the 128-byte-swizzled K-major stage: row r's 16-byte group j at byte
+        // r*128 + ((j ^ (r % 8)) * 16).
+        // The loads of the warp's next K block are issued before the current one is
+        // converted, so one load latency is exposed per warp, not one per K block.
+        const int qw = warp - 8;
+        constexpr int kItems = MP * 16 / 32;
+        auto load_block = [&](int i, uint4(&v)[kItems]) {
+            const int64_t colbase = static_cast<int64_t>(kb0 + i) * 128;
+#pragma unroll
+            for (int t = 0; t < kItems; ++t) {
+                const int item = lane + 32 * t;
+                const int r = item >> 4;
+                const int64_t col = colbase + (item & 15) * 8;
+                v[t] = make_uint4(0, 0, 0, 0);
+                if (i < nkb && r < p.M && col < p.K)  // K % 16 == 0: a group is whole or absent
+                    v[t] = p.Xa[(static_cast<int64_t>(r) * p.K + col) >> 3];
+            }
+        };
+        uint4 v[kItems], vn[kItems];
+        load_block(qw, v);
+        for (int i = qw; i < nkb; i += 4) {
             const int s = i % STAGES;
             const uint32_t u = static_cast<uint32_t>(i / STAGES);
-            const int ra = i % RA;
-            const uint32_t ua = static_cast<uint32_t>(i / RA);
-            // one thread waits for the slab and the stage and publishes the outcome,
-            // so that all 128 threads take the same path through the named barriers
-            if (qt == 0)
-                *stage_ok = (mbar_wait(&afull[ra], ua & 1u, abort_flag, p.timeout_ns) &&
-                             mbar_wait(&empty[s], (u & 1u) ^ 1u, abort_flag, p.timeout_ns))
-                                ? 1
-                                : 0;
-            bar_named_sync(2, 128);
-            if (!*stage_ok) {
-                if (qt == 0) {
+            const int64_t colbase = static_cast<int64_t>(kb0 + i) * 128;
+            load_block(i + 4, vn);
+            uint32_t m2 = 0;
+#pragma unroll
+            for (int t = 0; t < kItems; ++t) m2 = amax_fold8(m2, v[t]);
+            uint32_t ab = amax_bits_of(m2);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) ab = max(ab, __shfl_xor_sync(0xFFFFFFFFu, ab, o));
+            const BlockScale bs = block_scale(ab);
+            // the stage's previous K block has been consumed by its MMAs and its A
+            // scale read by the epilogue
+            int ok = 1;
+            if (lane == 0) ok = mbar_wait(&empty[s], (u & 1u) ^ 1u, abort_flag, p.timeout_ns) ? 1 : 0;
+            ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+            if (!ok) {
+                if (lane == 0) {
                     record_failure(p.status, kStatusTimeout, 13, i);
                     *abort_flag = 1;
                 }
                 break;
             }
-            // complete already (slot i % RA cannot refill before this slab is
-            // released): each reader acquires the TMA writes itself
-            mbar_wait(&afull[ra], ua & 1u, abort_flag, p.timeout_ns);
-            const uint8_t *slab = smem + L::kOffA + ra * L::kABytes;
-            const int64_t colbase = static_cast<int64_t>(kb0 + i) * 128;
-            uint4 v[kItems][2];
-            uint32_t m2 = 0;
-#pragma unroll
-            for (int t = 0; t < kItems; ++t) {
-                const int item = qt + t * 128;  // row item / 8, 16-column group item % 8
-                const uint4 *src = reinterpret_cast<const uint4 *>(slab + (item >> 3) * 256 + (item & 7) * 32);
-                v[t][0] = src[0];  // rows past M and columns past K arrive zero-filled
-                v[t][1] = src[1];
-                m2 = amax_fold8(amax_fold8(m2, v[t][0]), v[t][1]);
-            }
-            uint32_t ab = amax_bits_of(m2);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) ab = max(ab, __shfl_xor_sync(0xFFFFFFFFu, ab, o));
-            uint32_t *qr = qred + (i & 1) * 4;  // alternating halves: the previous round may still be read
-            if (lane == 0) qr[qw] = ab;
-            bar_named_sync(2, 128);
-            const BlockScale bs = block_scale(max(max(qr[0], qr[1]), max(qr[2], qr[3])));
             uint8_t *xs = smem + L::kOffX + s * L::kXBytes;
+            uint2 codes[kItems];
 #pragma unroll
             for (int t = 0; t < kItems; ++t) {
-                const int item = qt + t * 128;
-                const int r = item >> 3, j = item & 7;
-                const int64_t col = colbase + j * 16;
-                uint4 codes = make_uint4(0, 0, 0, 0);  // padding quantizes to +0
-                if (r < p.M && col < p.K) {             // K % 16 == 0: a group is whole or absent
-                    const uint2 lo = quantize8(v[t][0], bs), hi = quantize8(v[t][1], bs);
-                    codes = make_uint4(lo.x, lo.y, hi.x, hi.y);
-                    if (nb == 0) *reinterpret_cast<uint4 *>(p.qa_out + static_cast<int64_t>(r) * p.K + col) = codes;
-                }
-                *reinterpret_cast<uint4 *>(xs + r * 128 + ((j ^ (r & 7)) << 4)) = codes;
+                const int item = lane + 32 * t;
+                const int r = item >> 4, g = item & 15;
+                codes[t] = make_uint2(0, 0);
+                if (r < p.M && colbase + g * 8 < p.K) codes[t] = quantize8(v[t], bs);
+                *reinterpret_cast<uint2 *>(xs + r * 128 + (((g >> 1) ^ (r & 7)) << 4) + (g & 1) * 8) = codes[t];
             }
-            if (qt == 0) {
-                sa_stage[s] = bs.s;
-                if (nb == 0) p.sa_out[kb0 + i] = bs.s;
-            }
+            if (lane == 0) sa_stage[s] = bs.s;
             fence_async_smem();  // the codes are read by the tensor cores (async proxy)
-            bar_named_sync(2, 128);
-            if (qt == 0) {
-                mbar_arrive(&full[s]);
-                mbar_arrive(&aempty[ra]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&full[s]);
+            if (nb == 0) {  // the caller's copy, off the MMA's path
+#pragma unroll
+                for (int t = 0; t < kItems; ++t) {
+                    const int item = lane + 32 * t;
+                    const int r = item >> 4;
+                    const int64_t col = colbase + (item & 15) * 8;
+                    if (r < p.M && col < p.K)
+                        *reinterpret_cast<uint2 *>(p.qa_out + static_cast<int64_t>(r) * p.K + col) = codes[t];
+                }
+                if (lane == 0) p.sa_out[kb0 + i] = bs.s;
             }
+#pragma unroll
+            for (int t = 0; t < kItems; ++t) v[t] = vn[t];
         }
     } else if (warp >= 4 && warp < 8) {
         // -------------------------------------------------------------- epilogue
@@ -478,17 +443,14 @@ __global__ void __launch_bounds__(skinny_threads<FUSED>(), 1)
 template <int MP, int STAGES, int NBUF, bool FUSED>
 static dg_status_t launch_skinny_impl(const GemmArgs &a, const uint16_t *Xa, uint8_t *qa_out, float *sa_out,
                                       const DeviceInfo &dev, cudaStream_t stream) {
-    using L = SkinnySmem<MP, STAGES, NBUF, FUSED ? 4 : 0>;
+    using L = SkinnySmem<MP, STAGES, NBUF>;
     static_assert(L::kDynamicBytes <= 232448, "shared memory budget");
     CUtensorMap tmW, tmX;
     dg_status_t st = make_tmap_2d(&tmW, a.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.N, a.K, 128, 128,
                                   CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != DG_OK) return st;
     if (FUSED) {
-        // BF16 slabs of A: MP rows x 128 columns (256 bytes), unswizzled
-        st = make_tmap_2d(&tmX, Xa, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.M, a.K, MP, 128,
-                          CU_TENSOR_MAP_SWIZZLE_NONE);
-        if (st != DG_OK) return st;
+        tmX = tmW;  // unused: the quantizer warps read A from global memory
     } else {
         st = make_tmap_2d(&tmX, a.A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.M, a.K, MP, 128, CU_TENSOR_MAP_SWIZZLE_128B);
         if (st != DG_OK) return st;
@@ -523,7 +485,7 @@ static dg_status_t launch_skinny_impl(const GemmArgs &a, const uint16_t *Xa, uin
     p.timeout_ns = kernel_control().timeout_ns;
     p.status = kernel_control().status;
     p.debug_flags = kernel_control().debug_flags;
-    p.Xa = Xa;
+    p.Xa = reinterpret_cast<const uint4 *>(Xa);
     p.K = static_cast<int>(a.K);
     p.qa_out = qa_out;
     p.sa_out = sa_out;

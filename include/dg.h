@@ -123,10 +123,11 @@ dg_status_t dg_fp8_gemm_blockscaled(const uint8_t *A, const float *sA,
  *          Caller-owned: they receive A's codes and scales (the library allocates
  *          nothing).
  * Shapes as in dg_fp8_gemm_blockscaled (N % 16 == 0, K % 16 == 0, K > 0).
- * M == 1: one launch -- the skinny kernel quantizes A inside its producer
- * stage (no separate pass over A).  Larger M: the block quantizer, then the
- * FP8 GEMM, on `stream` (faster from M = 2 on, measured).  M == 0 or N == 0 is
- * a no-op.
+ * Runs the block quantizer, then dg_fp8_gemm_blockscaled's kernel, on `stream`;
+ * the quantizer lets the GEMM start its set-up and weight prefetch while it
+ * runs.  (The one-launch form, DG_KERNEL_SKINNY_FUSED in
+ * dg_fp8_gemm_blockscaled_bf16a_select, measured no faster for any M.)
+ * M == 0 or N == 0 is a no-op.
  */
 dg_status_t dg_fp8_gemm_blockscaled_bf16a(const void *A_bf16, const uint8_t *B, const float *sB,
                                           void *C_bf16, uint8_t *QA, float *sA,
@@ -222,12 +223,32 @@ dg_status_t dg_fp8_grouped_gemm_masked(const uint8_t *A, const float *sA,
  * TILE and PAIR run a last round that would leave at least half the SMs idle as
  * half-width tiles.
  */
-typedef enum { DG_KERNEL_AUTO = 0, DG_KERNEL_TILE = 1, DG_KERNEL_SKINNY = 2, DG_KERNEL_PAIR = 3 } dg_kernel_t;
+typedef enum {
+    DG_KERNEL_AUTO = 0,
+    DG_KERNEL_TILE = 1,
+    DG_KERNEL_SKINNY = 2,
+    DG_KERNEL_PAIR = 3,
+    DG_KERNEL_SKINNY_FUSED = 4 /* dg_fp8_gemm_blockscaled_bf16a_select only */
+} dg_kernel_t;
 
 dg_status_t dg_fp8_gemm_blockscaled_select(const uint8_t *A, const float *sA,
                                            const uint8_t *B, const float *sB, void *C_bf16,
                                            int64_t M, int64_t N, int64_t K,
                                            dg_kernel_t kernel, cudaStream_t stream);
+
+/*
+ * dg_fp8_gemm_blockscaled_bf16a with the kernel chosen, for tests and measurement.
+ * AUTO, TILE, SKINNY, PAIR: the block quantizer, then that GEMM kernel.
+ * SKINNY_FUSED (M <= 16, else DG_ERR_SHAPE): one launch of the skinny kernel,
+ * whose four extra warps quantize A's K blocks straight into the MMA's stages
+ * (same codes and scales, bit for bit; the CTAs of the first N block also write
+ * QA and sA).  2kiu.com/news/5461879 §5: activation scales are recomputed on
+ * every call.
+ */
+dg_status_t dg_fp8_gemm_blockscaled_bf16a_select(const void *A_bf16, const uint8_t *B, const float *sB,
+                                                 void *C_bf16, uint8_t *QA, float *sA,
+                                                 int64_t M, int64_t N, int64_t K,
+                                                 dg_kernel_t kernel, cudaStream_t stream);
 
 /* dg_fp8_gemm_1x128 with the kernel chosen: AUTO, TILE or PAIR (SKINNY gives
  * DG_ERR_INVALID_ARG), for tests and measurement. */
@@ -250,7 +271,8 @@ const char *dg_status_string(dg_status_t status);
 dg_status_t dg_get_last_device_status(cudaStream_t stream);
 
 /* Library ABI version (major * 100 + minor).  1.01 added the BF16-activation,
- * per-token-scale and masked-MoE calls; 1.02 added DG_ERR_GROUP_OFFSETS.  Every
+ * per-token-scale and masked-MoE calls; 1.02 added DG_ERR_GROUP_OFFSETS; 1.03
+ * added dg_fp8_gemm_blockscaled_bf16a_select and DG_KERNEL_SKINNY_FUSED.  Every
  * 1.00 call is unchanged. */
 int dg_version(void);
 

@@ -38,7 +38,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.dg_version() == 102
+    assert lib.dg_version() == 103
     for code, name in binding.STATUS_NAMES.items():
         assert lib.dg_status_string(code).decode().startswith(name)
     # the device-side group_offsets check has its own code, named in the header
@@ -99,6 +99,15 @@ def test_host_validation_without_device(lib):
     assert lib.dg_fp8_grouped_gemm_masked(odd, ok16, ok16, ok16, ok16, ok16, 2, 128, 128, 128, null) == 3
     # an unknown kernel choice
     assert lib.dg_fp8_gemm_1x128_select(ok16, ok16, ok16, ok16, ok16, 8, 16, 128, 9, null) == 1
+    # the fused one-launch form is a choice of the BF16-activation call only, up to M = 16
+    fused = 4
+    assert lib.dg_fp8_gemm_blockscaled_select(ok16, ok16, ok16, ok16, ok16, 8, 16, 128, fused, null) == 1
+    assert lib.dg_fp8_gemm_1x128_select(ok16, ok16, ok16, ok16, ok16, 8, 16, 128, fused, null) == 1
+    assert lib.dg_fp8_gemm_blockscaled_bf16a_select(ok16, ok16, ok16, ok16, ok16, ok16, 17, 16, 128, fused, null) == 2
+    assert lib.dg_fp8_gemm_blockscaled_bf16a_select(ok16, ok16, ok16, ok16, ok16, ok16, 200, 16, 128, 2, null) == 2
+    assert lib.dg_fp8_gemm_blockscaled_bf16a_select(ok16, ok16, ok16, ok16, ok16, ok16, 8, 16, 128, 9, null) == 1
+    assert lib.dg_fp8_gemm_blockscaled_bf16a_select(odd, ok16, ok16, ok16, ok16, ok16, 8, 16, 128, fused, null) == 3
+    assert lib.dg_fp8_gemm_blockscaled_bf16a_select(null, null, null, null, null, null, 0, 16, 128, fused, null) == 0
 
 
 def declared_signatures():

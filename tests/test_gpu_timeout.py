@@ -48,7 +48,7 @@ def test_skinny_cluster_kernel_times_out_cleanly(fused):
 
     def call():
         if fused:
-            return binding.gemm_blockscaled_bf16a(Abf, B, SB)[0]
+            return binding.gemm_blockscaled_bf16a(Abf, B, SB, kernel="fused")[0]
         return binding.gemm_blockscaled(A, SA, B, SB, kernel="skinny")
 
     assert binding.last_device_status() == 0
