@@ -379,17 +379,20 @@ __global__ void __launch_bounds__(kTileThreads, 1)
                 const uint32_t u = static_cast<uint32_t>(kc / STAGES);
                 const int buf = kc % NBUF;
                 const uint32_t v = static_cast<uint32_t>(kc / NBUF);
-                if (!mbar_wait(&tempty[buf], (v & 1u) ^ 1u, abort_flag, p.timeout_ns) ||
-                    !mbar_wait(&full[s], u & 1u, abort_flag, p.timeout_ns)) {
+                const uint64_t adesc = sdesc_kmajor_sw128(a0 + s * L::kABytes);
+                const uint64_t bdesc = sdesc_kmajor_sw128(b0 + s * L::kBBytes);
+                const uint32_t d = tmem_base + static_cast<uint32_t>(buf * BN);
+                const uint32_t idesc = narrow ? kIdescNarrow : kIdesc;
+                // The stage has almost always landed long before the buffer comes back
+                // from the epilogue: waiting on it first keeps its (successful) wait
+                // off the path from the hand-back to the first MMA.
+                if (!mbar_wait(&full[s], u & 1u, abort_flag, p.timeout_ns) ||
+                    !mbar_wait(&tempty[buf], (v & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
                     record_failure(p.status, kStatusTimeout, 1, kc);
                     *abort_flag = 1;
                     break;
                 }
                 tc_fence_after();
-                const uint64_t adesc = sdesc_kmajor_sw128(a0 + s * L::kABytes);
-                const uint64_t bdesc = sdesc_kmajor_sw128(b0 + s * L::kBBytes);
-                const uint32_t d = tmem_base + static_cast<uint32_t>(buf * BN);
-                const uint32_t idesc = narrow ? kIdescNarrow : kIdesc;
 #pragma unroll
                 for (int k = 0; k < 4; ++k)  // 32 bytes of K per instruction = +2 in the address field
                     umma_e4m3(d, adesc + 2u * k, bdesc + 2u * k, idesc, k > 0 ? 1u : 0u);
