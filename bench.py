@@ -91,6 +91,13 @@ def kernel_source_hash(fname: str) -> str:
     return h.hexdigest()[:16]
 
 
+def kernel_file_of(workload: str) -> str:
+    """Source file of the GEMM kernel the library dispatches for a workload: the skinny
+    split-K kernel for the M <= 128 workloads, the tile kernel for the rest (dense with
+    M > 128, grouped and masked MoE, per-token scales)."""
+    return "gemm_skinny.cu" if workload.startswith("skinny_m") else "gemm_tile.cu"
+
+
 def ncu_traffic(workload: str, kernel_file: str):
     return NCU_TRAFFIC.get((workload, kernel_file, kernel_source_hash(kernel_file)))
 
@@ -388,8 +395,7 @@ class Plan:
             self.cfg = dict(self.cfg, workload=name, a_scales="one per row and 128-K group (K-block-major)")
         self.skinny = not (self.grouped or self.masked or self.rowscale) and w.M <= 128
         self.fused = self.skinny and name.endswith("_fused")
-        self.kernel_file = ("gemm_tile.cu" if (self.grouped or self.masked)
-                            else "gemm_skinny.cu" if self.skinny else "gemm_pair.cu")
+        self.kernel_file = kernel_file_of(name)
         self.A_host = w.A.contiguous().reshape(rows_a, w.K)  # masked: the [G][M_max] slabs as rows
         self.A = self.A_host.to(dev)
         B = w.B.reshape(-1, w.K).to(dev) if (self.grouped or self.masked) else w.B.to(dev)
