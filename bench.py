@@ -69,6 +69,21 @@ SKINNY_GRAPH_STEPS = 240
 # keyed by workload, kernel file and the hash of that file's code; a kernel changed
 # since the capture reports null.
 NCU_TRAFFIC = {
+    # tile_gemm_kernel<256,kDense,4,2,0>, dense 4096^3 (1% outlier rows): 33.59 MB read + 2.39 MB written
+    ("dense_4096_outliers", "gemm_tile.cu", "50e052388b7a3f55"): 35981568,
+    # tile_gemm_kernel<256,kDense,4,2,0>, dense 8192^3: 463.21 MB read + 119.59 MB written
+    ("dense_8192", "gemm_tile.cu", "50e052388b7a3f55"): 582796288,
+    # tile_gemm_kernel<256,kContiguous,4,2,0>, 8 experts N=K=4096: 208.62 MB read + 118.08 MB written
+    ("moe_g8", "gemm_tile.cu", "50e052388b7a3f55"): 326695424,
+    # tile_gemm_kernel<256,kContiguous,4,2,0>, 64 experts N=2048 K=7168: 1383.13 MB read + 142.75 MB written
+    ("moe_g64_zipf", "gemm_tile.cu", "50e052388b7a3f55"): 1525877760,
+    # skinny_gemm_kernel<16,8,8,0> M=1 and M=16; <64,8,8,0> M=64; <128,6,4,0> M=128; <16,8,8,1> the
+    # one-launch fused M=1 (N=K=4096): B once, nothing written back to DRAM within the capture
+    ("skinny_m1", "gemm_skinny.cu", "32d3a058d2d4cc43"): 16813568,
+    ("skinny_m16", "gemm_skinny.cu", "32d3a058d2d4cc43"): 16875008,
+    ("skinny_m64", "gemm_skinny.cu", "32d3a058d2d4cc43"): 17073152,
+    ("skinny_m128", "gemm_skinny.cu", "32d3a058d2d4cc43"): 17336576,
+    ("skinny_m1_fused", "gemm_skinny.cu", "32d3a058d2d4cc43"): 16851200,
 }
 
 KERNEL_HEADERS = ("dg_device.cuh", "quant_e4m3.cuh", "dg_internal.h")  # device code the kernels include
