@@ -69,6 +69,8 @@ SKINNY_GRAPH_STEPS = 240
 # keyed by workload, kernel file and the hash of that file's code; a kernel changed
 # since the capture reports null.
 NCU_TRAFFIC = {
+    # tile_gemm_kernel<256,kDense,4,2,0>, dense 512^3 (16 half-tile units): 0.56 MB read, nothing written back
+    ("dense_512", "gemm_tile.cu", "50e052388b7a3f55"): 555008,
     # tile_gemm_kernel<256,kDense,4,2,0>, dense 4096^3 (1% outlier rows): 33.59 MB read + 2.39 MB written
     ("dense_4096_outliers", "gemm_tile.cu", "50e052388b7a3f55"): 35981568,
     # tile_gemm_kernel<256,kDense,4,2,0>, dense 8192^3: 463.21 MB read + 119.59 MB written

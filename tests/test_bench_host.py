@@ -27,7 +27,7 @@ def test_code_hash_ignores_comments_only(bench):
         assert bench.ncu_traffic(workload, fname) == traffic
         # keyed by the file of the kernel the bench looks up for that workload
         assert fname == bench.kernel_file_of(workload), (workload, fname)
-    assert bench.ncu_traffic("dense_512", "gemm_pair.cu") is None
+    assert bench.ncu_traffic("dense_512", "gemm_pair.cu") is None  # keyed by the dispatched kernel only
     assert bench.kernel_file_of("dense_8192") == "gemm_tile.cu"
     assert bench.kernel_file_of("moe_g64_zipf") == "gemm_tile.cu"
     assert bench.kernel_file_of("skinny_m1_fused") == "gemm_skinny.cu"
