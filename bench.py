@@ -81,11 +81,11 @@ NCU_TRAFFIC = {
     ("moe_g64_zipf", "gemm_tile.cu", "50e052388b7a3f55"): 1525877760,
     # skinny_gemm_kernel<16,8,8,0> M=1 and M=16; <64,8,8,0> M=64; <128,6,4,0> M=128; <16,8,8,1> the
     # one-launch fused M=1 (N=K=4096): B once, nothing written back to DRAM within the capture
-    ("skinny_m1", "gemm_skinny.cu", "32d3a058d2d4cc43"): 16813568,
-    ("skinny_m16", "gemm_skinny.cu", "32d3a058d2d4cc43"): 16875008,
-    ("skinny_m64", "gemm_skinny.cu", "32d3a058d2d4cc43"): 17073152,
-    ("skinny_m128", "gemm_skinny.cu", "32d3a058d2d4cc43"): 17336576,
-    ("skinny_m1_fused", "gemm_skinny.cu", "32d3a058d2d4cc43"): 16851200,
+    ("skinny_m1", "gemm_skinny.cu", "5e2810935f174f5c"): 16813568,
+    ("skinny_m16", "gemm_skinny.cu", "5e2810935f174f5c"): 16875264,
+    ("skinny_m64", "gemm_skinny.cu", "5e2810935f174f5c"): 17073664,
+    ("skinny_m128", "gemm_skinny.cu", "5e2810935f174f5c"): 17334016,
+    ("skinny_m1_fused", "gemm_skinny.cu", "5e2810935f174f5c"): 16851200,
 }
 
 KERNEL_HEADERS = ("dg_device.cuh", "quant_e4m3.cuh", "dg_internal.h")  # device code the kernels include

@@ -53,8 +53,14 @@ struct SkinnyParams {
     float *sa_out;
 };
 
-template <bool FUSED>
-constexpr int skinny_threads() { return FUSED ? 384 : 256; }
+// Epilogue warps: four (one per TMEM lane quarter), or for 128-row token slabs eight,
+// two per quarter each taking half the slab's columns, which halves the per-K-block
+// TMEM read and promotion (measured: M = 128 step 13.36 -> 13.13 us; at M = 64 the
+// extra warps cost more than they save, 9.60 -> 9.76 us).
+template <int MP, bool FUSED>
+constexpr int skinny_epi_warps() { return (!FUSED && MP == 128) ? 8 : 4; }
+template <int MP, bool FUSED>
+constexpr int skinny_threads() { return (FUSED || skinny_epi_warps<MP, FUSED>() == 8) ? 384 : 256; }
 
 __device__ __forceinline__ uint32_t cluster_rank() {
     uint32_t r;
@@ -120,10 +126,12 @@ __device__ __forceinline__ void cluster_sync_relaxed() {
 }
 
 template <int MP, int STAGES, int NBUF, bool FUSED>
-__global__ void __launch_bounds__(skinny_threads<FUSED>(), 1)
+__global__ void __launch_bounds__(skinny_threads<MP, FUSED>(), 1)
     skinny_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                        const SkinnyParams p) {
-    constexpr int kThreads = skinny_threads<FUSED>();
+    constexpr int kThreads = skinny_threads<MP, FUSED>();
+    constexpr int kEpiWarps = skinny_epi_warps<MP, FUSED>();
+    constexpr int kEpiCols = MP * 4 / kEpiWarps;  // token columns per epilogue warp
     using L = SkinnySmem<MP, STAGES, NBUF>;
     static_assert(STAGES % 2 == 0 && NBUF % 2 == 0, "each MMA thread must own its stages and buffers");
     constexpr uint32_t kTmemCols = tmem_cols_for(NBUF * MP);
@@ -166,7 +174,7 @@ __global__ void __launch_bounds__(skinny_threads<FUSED>(), 1)
         }
         for (int b = 0; b < NBUF; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 4);
+            mbar_init(&tempty[b], kEpiWarps);
         }
         for (int q = 0; q < 2; ++q) mbar_init(&mdone[q], 1);
         *abort_flag = 0;
@@ -327,13 +335,14 @@ __global__ void __launch_bounds__(skinny_threads<FUSED>(), 1)
 #pragma unroll
             for (int t = 0; t < kItems; ++t) v[t] = vn[t];
         }
-    } else if (warp >= 4 && warp < 8) {
+    } else if (warp >= 4 && warp < 4 + kEpiWarps) {
         // -------------------------------------------------------------- epilogue
         const int quarter = warp & 3;
+        const int col0 = ((warp - 4) >> 2) * kEpiCols;  // this warp's first token column
         const int row = quarter * 32 + lane;  // output column n = nb*128 + row
-        float2 acc[MP / 2];
+        float2 acc[kEpiCols / 2];
 #pragma unroll
-        for (int j = 0; j < MP / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
+        for (int j = 0; j < kEpiCols / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
         ScaleStream scales;
         scales.start(p.sA, p.sB + static_cast<int64_t>(nb) * p.Kb, kb0, kb1);
         for (int i = 0; i < nkb; ++i) {
@@ -364,8 +373,8 @@ __global__ void __launch_bounds__(skinny_threads<FUSED>(), 1)
             }
             const float2 s2 = make_float2(scale, scale);
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                                   static_cast<uint32_t>(buf * MP);
-            constexpr int kChunks = MP / 16;
+                                   static_cast<uint32_t>(buf * MP + col0);
+            constexpr int kChunks = kEpiCols / 16;
             uint32_t r0[16], r1[16];
             tmem_load16_async(taddr, r0);
             tmem_wait16(r0);
@@ -390,11 +399,11 @@ __global__ void __launch_bounds__(skinny_threads<FUSED>(), 1)
         // every MMA of this CTA has completed once the epilogue saw its last tfull
         // (or the MMA threads drained after a failure), so the stage memory may now
         // hold the partial tile, [MP][128]: consecutive threads write consecutive words
-        bar_named_sync(1, 128);  // the four epilogue warps: all TMEM reads done
+        bar_named_sync(1, 32 * kEpiWarps);  // every epilogue warp: all TMEM reads done
 #pragma unroll
-        for (int j = 0; j < MP / 2; ++j) {
-            red[(2 * j) * 128 + row] = acc[j].x;
-            red[(2 * j + 1) * 128 + row] = acc[j].y;
+        for (int j = 0; j < kEpiCols / 2; ++j) {
+            red[(col0 + 2 * j) * 128 + row] = acc[j].x;
+            red[(col0 + 2 * j + 1) * 128 + row] = acc[j].y;
         }
     }
 
@@ -492,7 +501,7 @@ static dg_status_t launch_skinny_impl(const GemmArgs &a, const uint16_t *Xa, uin
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(Nt * S), 1, 1);
-    cfg.blockDim = dim3(static_cast<unsigned>(skinny_threads<FUSED>()), 1, 1);
+    cfg.blockDim = dim3(static_cast<unsigned>(skinny_threads<MP, FUSED>()), 1, 1);
     cfg.dynamicSmemBytes = L::kDynamicBytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
