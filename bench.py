@@ -70,22 +70,22 @@ SKINNY_GRAPH_STEPS = 240
 # since the capture reports null.
 NCU_TRAFFIC = {
     # tile_gemm_kernel<256,kDense,4,2,0>, dense 512^3 (16 half-tile units): 0.56 MB read, nothing written back
-    ("dense_512", "gemm_tile.cu", "50e052388b7a3f55"): 555008,
-    # tile_gemm_kernel<256,kDense,4,2,0>, dense 4096^3 (1% outlier rows): 33.59 MB read + 2.39 MB written
-    ("dense_4096_outliers", "gemm_tile.cu", "50e052388b7a3f55"): 35981568,
-    # tile_gemm_kernel<256,kDense,4,2,0>, dense 8192^3: 463.21 MB read + 119.59 MB written
-    ("dense_8192", "gemm_tile.cu", "50e052388b7a3f55"): 582796288,
-    # tile_gemm_kernel<256,kContiguous,4,2,0>, 8 experts N=K=4096: 208.62 MB read + 118.08 MB written
-    ("moe_g8", "gemm_tile.cu", "50e052388b7a3f55"): 326695424,
-    # tile_gemm_kernel<256,kContiguous,4,2,0>, 64 experts N=2048 K=7168: 1383.13 MB read + 142.75 MB written
-    ("moe_g64_zipf", "gemm_tile.cu", "50e052388b7a3f55"): 1525877760,
+    ("dense_512", "gemm_tile.cu", "0963aafbf3ec9694"): 555520,
+    # tile_gemm_kernel<256,kDense,4,2,0>, dense 4096^3 (1% outlier rows): 33.59 MB read + 2.22 MB written
+    ("dense_4096_outliers", "gemm_tile.cu", "0963aafbf3ec9694"): 35816960,
+    # tile_gemm_kernel<256,kDense,4,2,0>, dense 8192^3: 451.30 MB read + 119.38 MB written
+    ("dense_8192", "gemm_tile.cu", "0963aafbf3ec9694"): 570679552,
+    # tile_gemm_kernel<256,kContiguous,4,2,0>, 8 experts N=K=4096: 209.60 MB read + 117.52 MB written
+    ("moe_g8", "gemm_tile.cu", "0963aafbf3ec9694"): 327121152,
+    # tile_gemm_kernel<256,kContiguous,4,2,0>, 64 experts N=2048 K=7168: 1405.11 MB read + 146.23 MB written
+    ("moe_g64_zipf", "gemm_tile.cu", "0963aafbf3ec9694"): 1551345152,
     # skinny_gemm_kernel<16,8,8,0> M=1 and M=16; <64,8,8,0> M=64; <128,6,4,0> M=128; <16,8,8,1> the
     # one-launch fused M=1 (N=K=4096): B once, nothing written back to DRAM within the capture
-    ("skinny_m1", "gemm_skinny.cu", "5e2810935f174f5c"): 16813568,
-    ("skinny_m16", "gemm_skinny.cu", "5e2810935f174f5c"): 16875264,
-    ("skinny_m64", "gemm_skinny.cu", "5e2810935f174f5c"): 17073664,
-    ("skinny_m128", "gemm_skinny.cu", "5e2810935f174f5c"): 17334016,
-    ("skinny_m1_fused", "gemm_skinny.cu", "5e2810935f174f5c"): 16851200,
+    ("skinny_m1", "gemm_skinny.cu", "e7452d79db77bcd8"): 16813824,
+    ("skinny_m16", "gemm_skinny.cu", "e7452d79db77bcd8"): 16875520,
+    ("skinny_m64", "gemm_skinny.cu", "e7452d79db77bcd8"): 17073664,
+    ("skinny_m128", "gemm_skinny.cu", "e7452d79db77bcd8"): 17334272,
+    ("skinny_m1_fused", "gemm_skinny.cu", "e7452d79db77bcd8"): 16851456,
 }
 
 KERNEL_HEADERS = ("dg_device.cuh", "quant_e4m3.cuh", "dg_internal.h")  # device code the kernels include

@@ -434,33 +434,6 @@ struct ScaleStream {
     }
 };
 
-// Wait with cluster-scope acquire (the arrivals come from the peer CTA too).
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, const volatile int *abort,
-                                                  uint64_t timeout_ns) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    uint32_t spins = 0;
-    while (true) {
-        if (mbar_try_wait_cluster(bar, parity)) return true;
-        if ((++spins & 31u) == 0) {
-            if (*abort) return false;
-            if (globaltimer_ns() - t0 > timeout_ns) return false;
-        }
-    }
-}
-
 // 2-D tiled TMA load into this CTA's shared memory whose byte count completes on
 // an mbarrier of either CTA of the pair (`bar_cluster` is a shared::cluster
 // address).  No multicast.
