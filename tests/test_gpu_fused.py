@@ -74,3 +74,37 @@ def test_bf16a_gemm_deterministic(M, kernel):
     outs = [binding.gemm_blockscaled_bf16a(A, B, SB, kernel=kernel)[0] for _ in range(3)]
     torch.cuda.synchronize()
     assert all(torch.equal(outs[0].view(torch.int16), o.view(torch.int16)) for o in outs[1:])
+
+
+@pytest.mark.parametrize("M,kernel", [(64, "skinny"), (200, "tile"), (200, "pair"), (16, "fused")])
+def test_bf16a_gemm_each_kernel_choice(M, kernel):
+    """Every kernel the BF16-activation call can be asked for gives the quantizer's codes
+    and scales bit for bit and C equal, bit for bit, to the FP8 GEMM of the same kernel
+    on those codes."""
+    N, K = 384, 640
+    d = inputs.dense_custom(M, N, K, seed=8900 + M)
+    qa_ref, sa_ref = oracle_quant(d.A)
+    qb, sb = oracle_quant(d.B)
+    B, SB = dev(qb), dev(sb)
+    C, QA, SA = binding.gemm_blockscaled_bf16a(d.A.cuda(), B, SB, kernel=kernel)
+    torch.cuda.synchronize()
+    assert binding.last_device_status() == 0
+    assert np.array_equal(QA.cpu().numpy(), qa_ref)
+    assert np.array_equal(SA.cpu().numpy().view(np.uint32), sa_ref.view(np.uint32))
+    C2 = binding.gemm_blockscaled(dev(qa_ref), dev(sa_ref), B, SB, kernel="skinny" if kernel == "fused" else kernel)
+    torch.cuda.synchronize()
+    assert torch.equal(C.view(torch.int16), C2.view(torch.int16))
+    check(c_f64(C), oracle.gemm_ref(qa_ref, sa_ref, qb, sb), None, f"bf16a {kernel} {M}x{N}x{K}")
+
+
+def test_bf16a_gemm_rejects_bad_kernel_choices():
+    A = torch.zeros((17, 128), dtype=torch.bfloat16, device="cuda")
+    B = torch.zeros((128, 128), dtype=torch.uint8, device="cuda")
+    SB = torch.ones((1, 1), dtype=torch.float32, device="cuda")
+    with pytest.raises(binding.DGError) as e:  # the one-launch form stops at 16 rows
+        binding.gemm_blockscaled_bf16a(A, B, SB, kernel="fused")
+    assert e.value.status == 2
+    with pytest.raises(binding.DGError) as e:  # the FP8-input GEMM has no fused form
+        binding.gemm_blockscaled(A.view(torch.uint8)[:, :128].contiguous(), torch.ones((1, 1), device="cuda"),
+                                 B, SB, kernel="fused")
+    assert e.value.status == 1
