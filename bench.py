@@ -79,6 +79,10 @@ NCU_TRAFFIC = {
     ("moe_g8", "gemm_tile.cu", "0963aafbf3ec9694"): 327121152,
     # tile_gemm_kernel<256,kContiguous,4,2,0>, 64 experts N=2048 K=7168: 1405.11 MB read + 146.23 MB written
     ("moe_g64_zipf", "gemm_tile.cu", "0963aafbf3ec9694"): 1551345152,
+    # tile_gemm_kernel<256,kDense,4,2,1> (one A scale per row and 128-K group), dense 4096^3: 34.13 MB read + 3.04 MB written
+    ("dense_4096_outliers_1x128", "gemm_tile.cu", "0963aafbf3ec9694"): 37164544,
+    # tile_gemm_kernel<256,kMasked,4,2,0>, 8 experts in 6912-row slabs, N=K=4096: 209.08 MB read + 114.98 MB written
+    ("moe_masked_g8", "gemm_tile.cu", "0963aafbf3ec9694"): 324064256,
     # skinny_gemm_kernel<16,8,8,0> M=1 and M=16; <64,8,8,0> M=64; <128,6,4,0> M=128; <16,8,8,1> the
     # one-launch fused M=1 (N=K=4096): B once, nothing written back to DRAM within the capture
     ("skinny_m1", "gemm_skinny.cu", "e7452d79db77bcd8"): 16813824,
@@ -134,8 +138,8 @@ WORKLOADS = ("dense_4096_outliers", "dense_512", "dense_8192", "skinny_m1", "ski
              "skinny_m128", "skinny_m1_fused", "skinny_m16_fused", "moe_g8", "moe_g64_zipf", "moe_masked_g8", "dense_4096_outliers_1x128",
              "moe_g64_zipf+dense_8192")
 # the default run: every benchmark workload, the last one on the top level
-SUITE = ("dense_512", "dense_4096_outliers", "skinny_m1", "skinny_m16", "skinny_m64", "skinny_m128", "moe_g8",
-         "moe_g64_zipf+dense_8192")
+SUITE = ("dense_512", "dense_4096_outliers", "dense_4096_outliers_1x128", "skinny_m1", "skinny_m1_fused",
+         "skinny_m16", "skinny_m64", "skinny_m128", "moe_g8", "moe_masked_g8", "moe_g64_zipf+dense_8192")
 TOP_LEVEL = "moe_g64_zipf+dense_8192"
 METRIC = "FP8 block-scaled GEMM TFLOPS (dense + MoE grouped) and % of B200 FP8 roofline"
 
@@ -452,8 +456,12 @@ class Plan:
             b.gemm_blockscaled(self.qa, self.sa, qb, sb, C=Cout)
 
     def quantize(self, x):
+        w = self.w
         if self.rowscale:
             self.b.quantize_1x128(x, q=self.qa, s_t=self.sa)
+        elif self.masked:  # only the slabs' token-holding blocks
+            self.b.quantize_blockwise_masked(x.view(w.G, w.M_max, w.K), self.mm, q=self.qa.view(w.G, w.M_max, w.K),
+                                             s=self.sa.view(w.G, w.M_max // 128, -1))
         else:
             self.b.quantize_blockwise(x, q=self.qa, s=self.sa)
 

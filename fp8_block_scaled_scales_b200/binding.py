@@ -23,7 +23,8 @@ STATUS_NAMES = {0: "DG_OK", 1: "DG_ERR_INVALID_ARG", 2: "DG_ERR_SHAPE", 3: "DG_E
 KERNELS = {"auto": 0, "tile": 1, "skinny": 2, "pair": 3, "fused": 4}
 
 # every symbol include/dg.h declares
-EXPORTS = ("dg_quantize_blockwise", "dg_fp8_gemm_blockscaled", "dg_fp8_gemm_blockscaled_bf16a",
+EXPORTS = ("dg_quantize_blockwise", "dg_quantize_blockwise_masked", "dg_fp8_gemm_blockscaled",
+           "dg_fp8_gemm_blockscaled_bf16a",
            "dg_fp8_gemm_blockscaled_bf16a_select",
            "dg_fp8_grouped_gemm_contiguous", "dg_fp8_grouped_gemm_masked", "dg_quantize_1x128",
            "dg_fp8_gemm_1x128", "dg_fp8_gemm_1x128_select",
@@ -51,6 +52,7 @@ def lib() -> ctypes.CDLL:
     L = ctypes.CDLL(LIB_PATH)
     vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
     L.dg_quantize_blockwise.argtypes = [vp, i64, i64, vp, vp, vp]
+    L.dg_quantize_blockwise_masked.argtypes = [vp, i32, i64, i64, vp, vp, vp, vp]
     L.dg_fp8_gemm_blockscaled.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp]
     L.dg_fp8_gemm_blockscaled_select.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, vp]
     L.dg_fp8_gemm_blockscaled_bf16a.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp]
@@ -60,7 +62,8 @@ def lib() -> ctypes.CDLL:
     L.dg_quantize_1x128.argtypes = [vp, i64, i64, vp, vp, vp]
     L.dg_fp8_gemm_1x128.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp]
     L.dg_fp8_gemm_1x128_select.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, vp]
-    for f in ("dg_quantize_blockwise", "dg_fp8_gemm_blockscaled", "dg_fp8_gemm_blockscaled_select",
+    for f in ("dg_quantize_blockwise", "dg_quantize_blockwise_masked", "dg_fp8_gemm_blockscaled",
+              "dg_fp8_gemm_blockscaled_select",
               "dg_fp8_gemm_blockscaled_bf16a", "dg_fp8_gemm_blockscaled_bf16a_select",
               "dg_fp8_grouped_gemm_contiguous", "dg_fp8_grouped_gemm_masked", "dg_get_last_device_status",
               "dg_quantize_1x128", "dg_fp8_gemm_1x128", "dg_fp8_gemm_1x128_select"):
@@ -113,6 +116,20 @@ def quantize_blockwise(x: torch.Tensor, q: torch.Tensor | None = None, s: torch.
         s = torch.empty(((R + 127) // 128, (C + 127) // 128), dtype=torch.float32, device=x.device)
     _check(lib().dg_quantize_blockwise(_p(x), R, C, _p(_u8(q)), _p(s), _stream(stream)),
            "dg_quantize_blockwise")
+    return q, s
+
+
+def quantize_blockwise_masked(x, masked_m, q=None, s=None, stream=None):
+    """Block quantization of masked-MoE activations x [G][M_max][K] (bf16): each slab as
+    quantize_blockwise would, except the 128-row blocks past masked_m[g] (int32 [G] on
+    the device), which are skipped (their codes and scales are not written)."""
+    G, M_max, K = x.shape
+    if q is None:
+        q = torch.zeros((G, M_max, K), dtype=torch.uint8, device=x.device)
+    if s is None:
+        s = torch.zeros((G, (M_max + 127) // 128, (K + 127) // 128), dtype=torch.float32, device=x.device)
+    _check(lib().dg_quantize_blockwise_masked(_p(x), G, M_max, K, _p(masked_m), _p(_u8(q)), _p(s), _stream(stream)),
+           "dg_quantize_blockwise_masked")
     return q, s
 
 

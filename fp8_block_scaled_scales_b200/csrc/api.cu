@@ -12,6 +12,12 @@
 
 namespace dg {
 
+// quantize.cu: `slabs` slabs of `rows` rows each, quantized slab by slab; with masked_m
+// (device, [slabs]) the row blocks of slab g at or past ceil(masked_m[g] / 128) are skipped.
+dg_status_t launch_quantize_masked(const void *X, int64_t slabs, int64_t rows, int64_t cols,
+                                   const int32_t *masked_m, uint8_t *Q, float *S, const DeviceInfo &dev,
+                                   cudaStream_t stream);
+
 // The device status word: [0] status of the first failure since the last read,
 // [1] role, [2] block, [3] step; [4..7] the snapshot the last read took.  One per
 // device (a module global).
@@ -153,7 +159,7 @@ using namespace dg;
 
 extern "C" {
 
-int dg_version(void) { return 103; }
+int dg_version(void) { return 104; }
 
 const char *dg_status_string(dg_status_t s) {
     switch (s) {
@@ -201,6 +207,18 @@ dg_status_t dg_quantize_blockwise(const void *X_bf16, int64_t rows, int64_t cols
     dg_status_t st = current_device(&dev, nullptr);
     if (st != DG_OK) return st;
     return launch_quantize(X_bf16, rows, cols, Q, S, dev, stream);
+}
+
+dg_status_t dg_quantize_blockwise_masked(const void *X_bf16, int G, int64_t M_max, int64_t cols,
+                                         const int32_t *masked_m, uint8_t *Q, float *S, cudaStream_t stream) {
+    if (G < 1 || G > 1024 || M_max < 0 || cols < 0 || cols % 16 != 0) return DG_ERR_SHAPE;
+    if (M_max == 0 || cols == 0) return DG_OK;
+    if (!X_bf16 || !masked_m || !Q || !S) return DG_ERR_INVALID_ARG;
+    if (!aligned(X_bf16, 16) || !aligned(Q, 16) || !aligned(S, 4) || !aligned(masked_m, 4)) return DG_ERR_ALIGNMENT;
+    DeviceInfo dev;
+    dg_status_t st = current_device(&dev, nullptr);
+    if (st != DG_OK) return st;
+    return launch_quantize_masked(X_bf16, G, M_max, cols, masked_m, Q, S, dev, stream);
 }
 
 dg_status_t dg_quantize_1x128(const void *X_bf16, int64_t rows, int64_t cols, uint8_t *Q, float *S_t,

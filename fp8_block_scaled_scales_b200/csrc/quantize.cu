@@ -27,17 +27,29 @@ constexpr int kQuantThreads = 256;
 
 // Four CTAs per SM (64 registers): measured 8 % faster than three on the 262 M-element
 // MoE activations (147.5 vs 160.1 us), the extra warps hiding load latency.
+// X is `slabs` slabs of R rows each, quantized slab by slab (a block never straddles
+// two slabs); block (g, lb, bc) is CTA (g * ceil(R/128) + lb) * Cb + bc and writes scale
+// S[that index].  masked_m (masked MoE, may be null): slab g's row blocks at or past
+// ceil(masked_m[g] / 128) hold no token and are skipped -- their Q and S are left as
+// they are; every other block is quantized exactly as without it.
 __global__ void __launch_bounds__(kQuantThreads, 4)
     quantize_kernel(const uint16_t *__restrict__ X, int64_t R, int64_t C, int64_t Cb, uint8_t *__restrict__ Q,
-                    float *__restrict__ S) {
+                    float *__restrict__ S, const int32_t *__restrict__ masked_m, int64_t Rb) {
     __shared__ uint32_t red[kQuantThreads / 32];
     // The GEMM that follows may start its set-up (and its weight prefetch into L2)
     // at once: it still waits for this grid to complete before reading Q and S.
     // Measured 5 % shorter for a quantize + skinny GEMM step at M = 16.
     grid_dep_launch_dependents();
-    grid_dep_wait();  // X may come from the previous kernel
+    grid_dep_wait();  // X (and masked_m) may come from the previous kernel
     const int64_t blk = blockIdx.x;
     const int64_t br = blk / Cb, bc = blk - br * Cb;
+    const int64_t g = br / Rb, lb = br - g * Rb;  // slab, row block inside it
+    if (masked_m != nullptr) {
+        const int64_t count = min(max(static_cast<int64_t>(__ldg(masked_m + g)), int64_t(0)), R);
+        if (lb * 128 >= count) return;  // no token in this block
+    }
+    const uint16_t *Xs = X + g * R * C;
+    uint8_t *Qs = Q + g * R * C;
     const int tid = static_cast<int>(threadIdx.x);
     const int chunk = tid & 15;  // 8-element column group
     const int sub = tid >> 4;    // 0..15
@@ -48,9 +60,9 @@ __global__ void __launch_bounds__(kQuantThreads, 4)
     uint32_t m2 = 0;  // two 16-bit magnitude maxima side by side
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const int64_t row = br * 128 + sub + 16 * i;
+        const int64_t row = lb * 128 + sub + 16 * i;
         if (col_ok && row < R) {
-            v[i] = __ldg(reinterpret_cast<const uint4 *>(X + row * C + col));
+            v[i] = __ldg(reinterpret_cast<const uint4 *>(Xs + row * C + col));
         } else {
             v[i] = make_uint4(0, 0, 0, 0);
         }
@@ -72,9 +84,9 @@ __global__ void __launch_bounds__(kQuantThreads, 4)
     if (!col_ok) return;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const int64_t row = br * 128 + sub + 16 * i;
+        const int64_t row = lb * 128 + sub + 16 * i;
         if (row >= R) break;
-        *reinterpret_cast<uint2 *>(Q + row * C + col) = quantize8(v[i], bs);
+        *reinterpret_cast<uint2 *>(Qs + row * C + col) = quantize8(v[i], bs);
     }
 }
 
@@ -116,14 +128,24 @@ dg_status_t launch_quantize_groups(const void *X, int64_t rows, int64_t cols, ui
                       static_cast<const uint16_t *>(X), rows, cols, Cb, groups, Q, St);
 }
 
+dg_status_t launch_quantize_masked(const void *X, int64_t slabs, int64_t rows, int64_t cols,
+                                   const int32_t *masked_m, uint8_t *Q, float *S, const DeviceInfo &dev,
+                                   cudaStream_t stream);
+
 dg_status_t launch_quantize(const void *X, int64_t rows, int64_t cols, uint8_t *Q, float *S,
                             const DeviceInfo &dev, cudaStream_t stream) {
+    return launch_quantize_masked(X, 1, rows, cols, nullptr, Q, S, dev, stream);
+}
+
+dg_status_t launch_quantize_masked(const void *X, int64_t slabs, int64_t rows, int64_t cols,
+                                   const int32_t *masked_m, uint8_t *Q, float *S, const DeviceInfo &dev,
+                                   cudaStream_t stream) {
     (void)dev;
     const int64_t Rb = (rows + 127) / 128, Cb = (cols + 127) / 128;
-    const int64_t blocks = Rb * Cb;
+    const int64_t blocks = slabs * Rb * Cb;
     if (blocks > 0x7FFFFFFFLL) return DG_ERR_SHAPE;
     return launch_pdl(quantize_kernel, static_cast<int>(blocks), kQuantThreads, 0, stream,
-                      static_cast<const uint16_t *>(X), rows, cols, Cb, Q, S);
+                      static_cast<const uint16_t *>(X), rows, cols, Cb, Q, S, masked_m, Rb);
 }
 
 }  // namespace dg

@@ -87,6 +87,28 @@ dg_status_t dg_quantize_blockwise(const void *X_bf16, int64_t rows, int64_t cols
                                   uint8_t *Q, float *S, cudaStream_t stream);
 
 /*
+ * dg_quantize_blockwise for the masked MoE layout (the activations of
+ * dg_fp8_grouped_gemm_masked): X holds G slabs of M_max rows, and slab g is
+ * quantized as dg_quantize_blockwise would quantize it alone (its blocks never reach
+ * into the next slab), except that its 128-row blocks at or past
+ * ceil(masked_m[g] / 128) -- the ones that hold no token -- are skipped: their
+ * codes and scales are not written.  Counts outside [0, M_max] are clamped.  The
+ * masked GEMM reads only the blocks written, so quantizing the slabs this way gives
+ * it the same inputs as quantizing them whole, for a fraction of the work when the
+ * slabs are mostly empty (2kiu.com/news/5461879 §2.2: only M varies between experts
+ * and it changes from call to call).
+ *
+ * X_bf16   : [G][M_max][cols] BF16, 16-byte aligned.
+ * masked_m : DEVICE int32 [G], 4-byte aligned (may be produced on `stream`).
+ * Q        : [G][M_max][cols] E4M3 out, 16-byte aligned.
+ * S        : [G][ceil(M_max/128)][ceil(cols/128)] FP32 out, 4-byte aligned.
+ * 1 <= G <= 1024, M_max >= 0, cols % 16 == 0.  M_max == 0 or cols == 0 is a no-op.
+ */
+dg_status_t dg_quantize_blockwise_masked(const void *X_bf16, int G, int64_t M_max, int64_t cols,
+                                         const int32_t *masked_m, uint8_t *Q_e4m3, float *S,
+                                         cudaStream_t stream);
+
+/*
  * Dense block-scaled GEMM, C = A * B^T (2kiu.com/news/5461879 §2.1, §3.3;
  * demingchina.com/news/60142 §3.1, §3.3):
  *   C[m][n] = bf16( sum_kb sA[m/128][kb] * sB[n/128][kb] *
@@ -272,8 +294,8 @@ dg_status_t dg_get_last_device_status(cudaStream_t stream);
 
 /* Library ABI version (major * 100 + minor).  1.01 added the BF16-activation,
  * per-token-scale and masked-MoE calls; 1.02 added DG_ERR_GROUP_OFFSETS; 1.03
- * added dg_fp8_gemm_blockscaled_bf16a_select and DG_KERNEL_SKINNY_FUSED.  Every
- * 1.00 call is unchanged. */
+ * added dg_fp8_gemm_blockscaled_bf16a_select and DG_KERNEL_SKINNY_FUSED; 1.04 added
+ * dg_quantize_blockwise_masked.  Every 1.00 call is unchanged. */
 int dg_version(void);
 
 /*

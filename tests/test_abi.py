@@ -38,7 +38,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.dg_version() == 103
+    assert lib.dg_version() == 104
     for code, name in binding.STATUS_NAMES.items():
         assert lib.dg_status_string(code).decode().startswith(name)
     # the device-side group_offsets check has its own code, named in the header
@@ -79,6 +79,12 @@ def test_host_validation_without_device(lib):
     assert lib.dg_fp8_grouped_gemm_masked(null, null, null, null, null, null, 2, 128, 128, 40, null) == 2
     assert lib.dg_fp8_grouped_gemm_masked(null, null, null, null, null, null, 2, 0, 128, 128, null) == 0
     assert lib.dg_fp8_grouped_gemm_masked(null, null, null, null, null, null, 2, 128, 128, 128, null) == 1
+    # masked-slab quantizer: G in [1, 1024], cols % 16, then pointers
+    assert lib.dg_quantize_blockwise_masked(null, 0, 128, 16, null, null, null, null) == 2
+    assert lib.dg_quantize_blockwise_masked(null, 1025, 128, 16, null, null, null, null) == 2
+    assert lib.dg_quantize_blockwise_masked(null, 2, 128, 17, null, null, null, null) == 2
+    assert lib.dg_quantize_blockwise_masked(null, 2, 0, 16, null, null, null, null) == 0
+    assert lib.dg_quantize_blockwise_masked(null, 2, 128, 16, null, null, null, null) == 1
     # per-token scales
     assert lib.dg_quantize_1x128(null, 4, 17, null, null, null) == 2
     assert lib.dg_quantize_1x128(null, 0, 16, null, null, null) == 0
@@ -91,6 +97,8 @@ def test_host_validation_without_device(lib):
     ok16 = ctypes.c_void_p(0x10000)
     assert lib.dg_quantize_blockwise(odd, 8, 16, ok16, ok16, null) == 3
     assert lib.dg_quantize_1x128(ok16, 8, 16, odd, ok16, null) == 3
+    assert lib.dg_quantize_blockwise_masked(ok16, 2, 8, 16, odd, ok16, ok16, null) == 3
+    assert lib.dg_quantize_blockwise_masked(odd, 2, 8, 16, ok16, ok16, ok16, null) == 3
     assert lib.dg_fp8_gemm_blockscaled_bf16a(odd, ok16, ok16, ok16, ok16, ok16, 8, 16, 128, null) == 3
     assert lib.dg_fp8_gemm_blockscaled_bf16a(ok16, ok16, ok16, ok16, odd, ok16, 8, 16, 128, null) == 3
     assert lib.dg_fp8_gemm_1x128(ok16, ok16, odd, ok16, ok16, 8, 16, 128, null) == 3

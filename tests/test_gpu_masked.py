@@ -124,3 +124,47 @@ def test_masked_largest_expert_count():
     check(got, real, float(np.sqrt(np.mean(real ** 2))), "masked G=256")
     for g in range(G):
         assert np.all(C[g, counts[g]:] == -3.0)
+
+
+@pytest.mark.parametrize("G,Mmax,K,counts", [
+    (4, 200, 256, [0, 200, 77, 129]),        # an empty slab, a full one, partial last blocks
+    (3, 384, 4000, [384, 1, 128]),           # K tail; a block boundary exactly at the count
+    (2, 130, 144, [-5, 1000]),               # counts clamped to [0, M_max]
+])
+def test_masked_quantizer_writes_the_token_blocks_exactly(G, Mmax, K, counts):
+    """Each slab's token-holding 128-row blocks get the block quantizer's codes and
+    scales bit for bit; the blocks past the count keep whatever the buffers held."""
+    w = inputs.masked_custom(G, Mmax, 128, K, np.clip(counts, 0, Mmax), seed=9300 + G + K)
+    qa_ref, sa_ref = oracle_quant(w.A)
+    mm = torch.from_numpy(np.asarray(counts, dtype=np.int32)).cuda()
+    Q = torch.full((G, Mmax, K), 0xA5, dtype=torch.uint8, device="cuda")
+    S = torch.full((G, (Mmax + 127) // 128, (K + 127) // 128), -7.0, dtype=torch.float32, device="cuda")
+    binding.quantize_blockwise_masked(w.A.cuda(), mm, q=Q, s=S)
+    torch.cuda.synchronize()
+    assert binding.last_device_status() == 0
+    Qh, Sh = Q.cpu().numpy(), S.cpu().numpy()
+    for g in range(G):
+        c = min(max(counts[g], 0), Mmax)
+        nb = (c + 127) // 128                    # blocks holding a token
+        rows = min(nb * 128, Mmax)
+        assert np.array_equal(Qh[g, :rows], qa_ref[g, :rows]), f"slab {g}: codes"
+        assert np.array_equal(Sh[g, :nb].view(np.uint32), sa_ref[g, :nb].view(np.uint32)), f"slab {g}: scales"
+        assert np.all(Qh[g, rows:] == 0xA5) and np.all(Sh[g, nb:] == -7.0), f"slab {g}: skipped blocks written"
+
+
+def test_masked_quantizer_feeds_the_masked_gemm_like_the_whole_quantizer():
+    """The masked GEMM on the slab-skipping quantizer's output equals, bit for bit, the
+    masked GEMM on the whole-slab quantizer's output."""
+    G, Mmax, N, K, counts = 4, 512, 256, 512, [300, 0, 129, 512]
+    w = inputs.masked_custom(G, Mmax, N, K, counts, seed=9400)
+    qb, sb = oracle_quant(w.B)
+    mm = torch.from_numpy(np.asarray(counts, dtype=np.int32)).cuda()
+    A = w.A.cuda()
+    qa1, sa1 = binding.quantize_blockwise_masked(A, mm)
+    qa2, sa2 = binding.quantize_blockwise(A.view(G * Mmax, K))
+    C1 = binding.grouped_gemm_masked(qa1, sa1, dev(qb), dev(sb), mm)
+    C2 = binding.grouped_gemm_masked(qa2.view(G, Mmax, K), sa2.view(G, Mmax // 128, -1), dev(qb), dev(sb), mm)
+    torch.cuda.synchronize()
+    assert binding.last_device_status() == 0
+    for g in range(G):
+        assert torch.equal(C1[g, :counts[g]].view(torch.int16), C2[g, :counts[g]].view(torch.int16))
