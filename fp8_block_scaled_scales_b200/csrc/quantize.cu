@@ -27,11 +27,12 @@ constexpr int kQuantThreads = 256;
 
 // Four CTAs per SM (64 registers): measured 8 % faster than three on the 262 M-element
 // MoE activations (147.5 vs 160.1 us), the extra warps hiding load latency.
-// X is `slabs` slabs of R rows each, quantized slab by slab (a block never straddles
-// two slabs); block (g, lb, bc) is CTA (g * ceil(R/128) + lb) * Cb + bc and writes scale
-// S[that index].  masked_m (masked MoE, may be null): slab g's row blocks at or past
-// ceil(masked_m[g] / 128) hold no token and are skipped -- their Q and S are left as
-// they are; every other block is quantized exactly as without it.
+// MASKED: X is slabs of R rows each, quantized slab by slab (a block never straddles
+// two slabs); block (g, lb, bc) is CTA (g * Rb + lb) * Cb + bc and writes scale
+// S[that index]; slab g's row blocks at or past ceil(masked_m[g] / 128) hold no token
+// and are skipped -- their Q and S are left as they are; every other block is
+// quantized exactly as without the mask.  Otherwise one matrix of R rows.
+template <bool MASKED>
 __global__ void __launch_bounds__(kQuantThreads, 4)
     quantize_kernel(const uint16_t *__restrict__ X, int64_t R, int64_t C, int64_t Cb, uint8_t *__restrict__ Q,
                     float *__restrict__ S, const int32_t *__restrict__ masked_m, int64_t Rb) {
@@ -43,8 +44,8 @@ __global__ void __launch_bounds__(kQuantThreads, 4)
     grid_dep_wait();  // X (and masked_m) may come from the previous kernel
     const int64_t blk = blockIdx.x;
     const int64_t br = blk / Cb, bc = blk - br * Cb;
-    const int64_t g = br / Rb, lb = br - g * Rb;  // slab, row block inside it
-    if (masked_m != nullptr) {
+    const int64_t g = MASKED ? br / Rb : 0, lb = MASKED ? br - g * Rb : br;  // slab, row block inside it
+    if (MASKED) {
         const int64_t count = min(max(static_cast<int64_t>(__ldg(masked_m + g)), int64_t(0)), R);
         if (lb * 128 >= count) return;  // no token in this block
     }
@@ -144,8 +145,11 @@ dg_status_t launch_quantize_masked(const void *X, int64_t slabs, int64_t rows, i
     const int64_t Rb = (rows + 127) / 128, Cb = (cols + 127) / 128;
     const int64_t blocks = slabs * Rb * Cb;
     if (blocks > 0x7FFFFFFFLL) return DG_ERR_SHAPE;
-    return launch_pdl(quantize_kernel, static_cast<int>(blocks), kQuantThreads, 0, stream,
-                      static_cast<const uint16_t *>(X), rows, cols, Cb, Q, S, masked_m, Rb);
+    if (masked_m == nullptr && slabs != 1) return DG_ERR_INVALID_ARG;
+    return masked_m ? launch_pdl(quantize_kernel<true>, static_cast<int>(blocks), kQuantThreads, 0, stream,
+                                 static_cast<const uint16_t *>(X), rows, cols, Cb, Q, S, masked_m, Rb)
+                    : launch_pdl(quantize_kernel<false>, static_cast<int>(blocks), kQuantThreads, 0, stream,
+                                 static_cast<const uint16_t *>(X), rows, cols, Cb, Q, S, masked_m, Rb);
 }
 
 }  // namespace dg
