@@ -278,13 +278,13 @@ def oracle_sample(w, rows_sample: int, seed: int = 0, rowscale: bool = False):
     from fp8_block_scaled_scales_b200 import inputs
     from fp8_block_scaled_scales_b200.inputs import Grouped, Masked
     if isinstance(w, Masked):
-        # the expert with the most tokens: its first rows_sample tokens (whole 128-row blocks)
+        # the expert with the most tokens: its first rows_sample tokens (whole 128-row
+        # blocks, or all of its tokens), quantized as the masked quantizer does
         g = int(np.argmax(w.counts))
         qb, sb = oracle.quantize_blockwise(inputs.bf16_bits(w.B[g]))
         rows = int(min(int(w.counts[g]), max(1, rows_sample // 128) * 128))
-        nblk = -(-rows // 128)
         t0 = time.perf_counter()
-        qa, sa = oracle.quantize_blockwise(inputs.bf16_bits(w.A[g, :nblk * 128]))
+        qa, sa = oracle.quantize_blockwise(inputs.bf16_bits(w.A[g, :rows]))
         ref = oracle.gemm_ref(qa, sa, qb, sb, rows=np.arange(rows))
         out = oracle.bf16_from_double(ref)
         dt = time.perf_counter() - t0
@@ -419,6 +419,9 @@ class Plan:
         self.kernel_file = kernel_file_of(name)
         self.A_host = w.A.contiguous().reshape(rows_a, w.K)  # masked: the [G][M_max] slabs as rows
         self.A = self.A_host.to(dev)
+        # (first row, rows) of A and C that carry the step's data: a masked slab's tokens only
+        self.io_rows = ([(g * w.M_max, int(w.counts[g])) for g in range(w.G) if w.counts[g]] if self.masked
+                        else [(0, rows_a)])
         B = w.B.reshape(-1, w.K).to(dev) if (self.grouped or self.masked) else w.B.to(dev)
         self.qb, self.sb = binding.quantize_blockwise(B)  # cached weights
         del B
@@ -533,26 +536,38 @@ def graph_step_ms(step_i, n_steps, reps, flush):
 
 def e2e_ms(plans, steps, stream):
     """Per-step ms through the C ABI with host buffers: every step copies its
-    activations in from pinned host memory and its C out to pinned host memory.  As
+    activations in from pinned host memory and its C out to pinned host memory (the
+    rows that carry data: of a masked slab, its tokens, whose results depend on
+    nothing past them).  As
     a serving loop would, the copies of neighbouring steps overlap the compute when
     they are large (two device staging buffers, three streams ordered by events);
     small steps run copy in, step, copy out on one stream."""
     A_pin = [p.A_host.pin_memory() for p in plans]
     C_pin = [[torch.empty(tuple(p.C.shape), dtype=torch.bfloat16).pin_memory() for p in plans] for _ in range(2)]
-    A_stage = [[torch.empty_like(p.A) for p in plans] for _ in range(2)]
+    A_stage = [[p.A.clone() for p in plans] for _ in range(2)]
     C_dev = [[p.C for p in plans], [torch.empty_like(p.C) for p in plans]]
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
     comp_done, out_done = [None, None], [None, None]
-    io_bytes = sum(p.A_host.numel() * 2 + p.C.numel() * 2 for p in plans)
-    pipelined = io_bytes >= E2E_PIPELINE_MIN_BYTES
+    h2d = sum(n * p.A.shape[1] * 2 for p in plans for _, n in p.io_rows)
+    d2h = sum(n * p.C.shape[1] * 2 for p in plans for _, n in p.io_rows)
+    pipelined = h2d + d2h >= E2E_PIPELINE_MIN_BYTES
+
+    def copy_in(b):
+        for k, p in enumerate(plans):
+            for r0, n in p.io_rows:
+                A_stage[b][k][r0:r0 + n].copy_(A_pin[k][r0:r0 + n], non_blocking=True)
+
+    def copy_out(b):
+        for k, p in enumerate(plans):
+            for r0, n in p.io_rows:
+                C_pin[b][k][r0:r0 + n].copy_(C_dev[b][k][r0:r0 + n], non_blocking=True)
 
     def step_pipe(i):
         b = i % 2
         with torch.cuda.stream(s_in):
             if comp_done[b] is not None:
                 s_in.wait_event(comp_done[b])  # staging buffer b has been read
-            for k in range(len(plans)):
-                A_stage[b][k].copy_(A_pin[k], non_blocking=True)
+            copy_in(b)
             ev_in = torch.cuda.Event()
             ev_in.record(s_in)
         stream.wait_event(ev_in)
@@ -564,16 +579,15 @@ def e2e_ms(plans, steps, stream):
         comp_done[b].record(stream)
         with torch.cuda.stream(s_out):
             s_out.wait_event(comp_done[b])
-            for k in range(len(plans)):
-                C_pin[b][k].copy_(C_dev[b][k], non_blocking=True)
+            copy_out(b)
             out_done[b] = torch.cuda.Event()
             out_done[b].record(s_out)
 
     def step_serial(i):
+        copy_in(0)
         for k, p in enumerate(plans):
-            A_stage[0][k].copy_(A_pin[k], non_blocking=True)
             p.step(A_stage[0][k], C_dev[0][k])
-            C_pin[0][k].copy_(C_dev[0][k], non_blocking=True)
+        copy_out(0)
 
     run = step_pipe if pipelined else step_serial
     for i in range(2):
@@ -591,8 +605,6 @@ def e2e_ms(plans, steps, stream):
     torch.cuda.synchronize()
     mode = ("copies of neighbouring steps overlap the compute (2 staging buffers, 3 streams)" if pipelined
             else "copy in, step, copy out on one stream")
-    h2d = sum(p.A_host.numel() * 2 for p in plans)
-    d2h = sum(p.C.numel() * 2 for p in plans)
     del A_pin, C_pin, A_stage, C_dev
     return e0.elapsed_time(e1) / steps, mode, h2d, d2h
 

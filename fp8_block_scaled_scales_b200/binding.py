@@ -120,9 +120,10 @@ def quantize_blockwise(x: torch.Tensor, q: torch.Tensor | None = None, s: torch.
 
 
 def quantize_blockwise_masked(x, masked_m, q=None, s=None, stream=None):
-    """Block quantization of masked-MoE activations x [G][M_max][K] (bf16): each slab as
-    quantize_blockwise would, except the 128-row blocks past masked_m[g] (int32 [G] on
-    the device), which are skipped (their codes and scales are not written)."""
+    """Block quantization of masked-MoE activations x [G][M_max][K] (bf16): the first
+    masked_m[g] rows of slab g (int32 [G] on the device) as quantize_blockwise would
+    quantize them alone; rows past the count and the blocks past the last token are
+    neither read nor written."""
     G, M_max, K = x.shape
     if q is None:
         q = torch.zeros((G, M_max, K), dtype=torch.uint8, device=x.device)

@@ -27,11 +27,12 @@ constexpr int kQuantThreads = 256;
 
 // Four CTAs per SM (64 registers): measured 8 % faster than three on the 262 M-element
 // MoE activations (147.5 vs 160.1 us), the extra warps hiding load latency.
-// MASKED: X is slabs of R rows each, quantized slab by slab (a block never straddles
-// two slabs); block (g, lb, bc) is CTA (g * Rb + lb) * Cb + bc and writes scale
-// S[that index]; slab g's row blocks at or past ceil(masked_m[g] / 128) hold no token
-// and are skipped -- their Q and S are left as they are; every other block is
-// quantized exactly as without the mask.  Otherwise one matrix of R rows.
+// MASKED: X is slabs of R rows each; slab g holds masked_m[g] tokens (clamped to
+// [0, R]) in its first rows and is quantized as the matrix of those rows alone: the
+// last token block's amax covers its tokens only, rows past the count are neither
+// read nor written, and the blocks past the last token are skipped (their Q and S
+// are left as they are).  Block (g, lb, bc) is CTA (g * Rb + lb) * Cb + bc and
+// writes scale S[that index].  Otherwise one matrix of R rows.
 template <bool MASKED>
 __global__ void __launch_bounds__(kQuantThreads, 4)
     quantize_kernel(const uint16_t *__restrict__ X, int64_t R, int64_t C, int64_t Cb, uint8_t *__restrict__ Q,
@@ -45,10 +46,9 @@ __global__ void __launch_bounds__(kQuantThreads, 4)
     const int64_t blk = blockIdx.x;
     const int64_t br = blk / Cb, bc = blk - br * Cb;
     const int64_t g = MASKED ? br / Rb : 0, lb = MASKED ? br - g * Rb : br;  // slab, row block inside it
-    if (MASKED) {
-        const int64_t count = min(max(static_cast<int64_t>(__ldg(masked_m + g)), int64_t(0)), R);
-        if (lb * 128 >= count) return;  // no token in this block
-    }
+    // rows of this matrix: the slab's tokens when masked
+    const int64_t rows = MASKED ? min(max(static_cast<int64_t>(__ldg(masked_m + g)), int64_t(0)), R) : R;
+    if (MASKED && lb * 128 >= rows) return;  // no token in this block
     const uint16_t *Xs = X + g * R * C;
     uint8_t *Qs = Q + g * R * C;
     const int tid = static_cast<int>(threadIdx.x);
@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(kQuantThreads, 4)
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int64_t row = lb * 128 + sub + 16 * i;
-        if (col_ok && row < R) {
+        if (col_ok && row < rows) {
             v[i] = __ldg(reinterpret_cast<const uint4 *>(Xs + row * C + col));
         } else {
             v[i] = make_uint4(0, 0, 0, 0);
@@ -86,7 +86,7 @@ __global__ void __launch_bounds__(kQuantThreads, 4)
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int64_t row = lb * 128 + sub + 16 * i;
-        if (row >= R) break;
+        if (row >= rows) break;
         *reinterpret_cast<uint2 *>(Qs + row * C + col) = quantize8(v[i], bs);
     }
 }

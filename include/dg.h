@@ -88,15 +88,16 @@ dg_status_t dg_quantize_blockwise(const void *X_bf16, int64_t rows, int64_t cols
 
 /*
  * dg_quantize_blockwise for the masked MoE layout (the activations of
- * dg_fp8_grouped_gemm_masked): X holds G slabs of M_max rows, and slab g is
- * quantized as dg_quantize_blockwise would quantize it alone (its blocks never reach
- * into the next slab), except that its 128-row blocks at or past
- * ceil(masked_m[g] / 128) -- the ones that hold no token -- are skipped: their
- * codes and scales are not written.  Counts outside [0, M_max] are clamped.  The
- * masked GEMM reads only the blocks written, so quantizing the slabs this way gives
- * it the same inputs as quantizing them whole, for a fraction of the work when the
- * slabs are mostly empty (2kiu.com/news/5461879 §2.2: only M varies between experts
- * and it changes from call to call).
+ * dg_fp8_grouped_gemm_masked): X holds G slabs of M_max rows, slab g holds
+ * masked_m[g] tokens in its first rows (counts outside [0, M_max] are clamped),
+ * and each slab's tokens are quantized as dg_quantize_blockwise would quantize the
+ * masked_m[g]-row matrix of them alone: the amax of the last token block covers
+ * its tokens only, rows past the count are neither read nor written, and the
+ * 128-row blocks at or past ceil(masked_m[g] / 128) are skipped (their scales are
+ * not written).  So no code or scale depends on the rows past a count, which may
+ * hold anything, and the work follows the tokens, not the slabs
+ * (2kiu.com/news/5461879 §2.2: only M varies between experts and it changes from
+ * call to call).
  *
  * X_bf16   : [G][M_max][cols] BF16, 16-byte aligned.
  * masked_m : DEVICE int32 [G], 4-byte aligned (may be produced on `stream`).

@@ -17,6 +17,21 @@ def oracle_quant(x_bf16: torch.Tensor):
     return oracle.quantize_blockwise(inputs.bf16_bits(x_bf16))
 
 
+def oracle_quant_tokens(x_bf16: torch.Tensor, counts):
+    """Oracle quantization of masked-MoE activations [G][M_max][K]: the first counts[g]
+    rows of slab g quantized as a matrix of their own.  Codes of the rows past a count
+    are 0 and the scales of the blocks past the last token 1 (no output reads them)."""
+    G, M_max, K = x_bf16.shape
+    qa = np.zeros((G, M_max, K), np.uint8)
+    sa = np.ones((G, -(-M_max // 128), -(-K // 128)), np.float32)
+    for g in range(G):
+        c = min(max(int(counts[g]), 0), M_max)
+        if c:
+            q, s = oracle.quantize_blockwise(inputs.bf16_bits(x_bf16[g, :c]))
+            qa[g, :c], sa[g, :s.shape[0]] = q, s
+    return qa, sa
+
+
 def dev(a: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(a)).cuda()
 

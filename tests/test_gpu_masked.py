@@ -6,13 +6,13 @@ import torch
 import oracle
 from fp8_block_scaled_scales_b200 import binding, inputs
 
-from parity import c_f64, check, dev, oracle_quant
+from parity import c_f64, check, dev, oracle_quant, oracle_quant_tokens
 
 pytestmark = pytest.mark.gpu
 
 
 def quantized(w, junk_seed=None):
-    qa, sa = oracle_quant(w.A)   # per expert slab: [G][M_max][K], [G][ceil(M_max/128)][Kb]
+    qa, sa = oracle_quant_tokens(w.A, w.counts)  # [G][M_max][K], [G][ceil(M_max/128)][Kb]
     qb, sb = oracle_quant(w.B)
     if junk_seed is not None:
         # rows past each count may hold anything, NaN codes included: no output may see them
@@ -131,11 +131,13 @@ def test_masked_largest_expert_count():
     (3, 384, 4000, [384, 1, 128]),           # K tail; a block boundary exactly at the count
     (2, 130, 144, [-5, 1000]),               # counts clamped to [0, M_max]
 ])
-def test_masked_quantizer_writes_the_token_blocks_exactly(G, Mmax, K, counts):
-    """Each slab's token-holding 128-row blocks get the block quantizer's codes and
-    scales bit for bit; the blocks past the count keep whatever the buffers held."""
-    w = inputs.masked_custom(G, Mmax, 128, K, np.clip(counts, 0, Mmax), seed=9300 + G + K)
-    qa_ref, sa_ref = oracle_quant(w.A)
+def test_masked_quantizer_quantizes_each_slabs_tokens_alone(G, Mmax, K, counts):
+    """Slab g's first counts[g] rows get, bit for bit, the block quantizer's codes and
+    scales for the matrix of those rows alone (its last block's amax covers tokens
+    only); rows past the count and blocks past the last token keep what the buffers held."""
+    clamped = np.clip(counts, 0, Mmax)
+    w = inputs.masked_custom(G, Mmax, 128, K, clamped, seed=9300 + G + K)
+    qa_ref, sa_ref = oracle_quant_tokens(w.A, clamped)
     mm = torch.from_numpy(np.asarray(counts, dtype=np.int32)).cuda()
     Q = torch.full((G, Mmax, K), 0xA5, dtype=torch.uint8, device="cuda")
     S = torch.full((G, (Mmax + 127) // 128, (K + 127) // 128), -7.0, dtype=torch.float32, device="cuda")
@@ -144,26 +146,50 @@ def test_masked_quantizer_writes_the_token_blocks_exactly(G, Mmax, K, counts):
     assert binding.last_device_status() == 0
     Qh, Sh = Q.cpu().numpy(), S.cpu().numpy()
     for g in range(G):
-        c = min(max(counts[g], 0), Mmax)
+        c = int(clamped[g])
         nb = (c + 127) // 128                    # blocks holding a token
-        rows = min(nb * 128, Mmax)
-        assert np.array_equal(Qh[g, :rows], qa_ref[g, :rows]), f"slab {g}: codes"
+        assert np.array_equal(Qh[g, :c], qa_ref[g, :c]), f"slab {g}: codes"
         assert np.array_equal(Sh[g, :nb].view(np.uint32), sa_ref[g, :nb].view(np.uint32)), f"slab {g}: scales"
-        assert np.all(Qh[g, rows:] == 0xA5) and np.all(Sh[g, nb:] == -7.0), f"slab {g}: skipped blocks written"
+        assert np.all(Qh[g, c:] == 0xA5) and np.all(Sh[g, nb:] == -7.0), f"slab {g}: rows past the count written"
 
 
-def test_masked_quantizer_feeds_the_masked_gemm_like_the_whole_quantizer():
-    """The masked GEMM on the slab-skipping quantizer's output equals, bit for bit, the
-    masked GEMM on the whole-slab quantizer's output."""
+def test_masked_quantizer_ignores_rows_past_the_count():
+    """Changing the rows past each count (to anything, infinities and NaN included)
+    changes no code or scale the quantizer writes."""
+    G, Mmax, K, counts = 3, 256, 384, [77, 128, 200]
+    w = inputs.masked_custom(G, Mmax, 128, K, counts, seed=9350)
+    mm = torch.tensor(counts, dtype=torch.int32, device="cuda")
+    A = w.A.cuda()
+    q1, s1 = binding.quantize_blockwise_masked(A, mm)
+    A2 = A.clone()
+    rng = np.random.default_rng(9351)
+    for g in range(G):
+        junk = rng.integers(0, 1 << 16, size=(Mmax - counts[g], K), dtype=np.uint16)
+        A2[g, counts[g]:] = torch.from_numpy(junk.view(np.int16)).cuda().view(torch.bfloat16)
+    q2, s2 = binding.quantize_blockwise_masked(A2, mm)
+    torch.cuda.synchronize()
+    assert binding.last_device_status() == 0
+    assert torch.equal(q1, q2) and torch.equal(s1.view(torch.int32), s2.view(torch.int32))
+
+
+def test_masked_quantizer_feeds_the_masked_gemm_like_per_expert_quantization():
+    """The masked GEMM on the masked quantizer's output equals, bit for bit, the masked
+    GEMM on each expert's tokens quantized by the plain quantizer as a matrix of their own."""
     G, Mmax, N, K, counts = 4, 512, 256, 512, [300, 0, 129, 512]
     w = inputs.masked_custom(G, Mmax, N, K, counts, seed=9400)
     qb, sb = oracle_quant(w.B)
     mm = torch.from_numpy(np.asarray(counts, dtype=np.int32)).cuda()
     A = w.A.cuda()
     qa1, sa1 = binding.quantize_blockwise_masked(A, mm)
-    qa2, sa2 = binding.quantize_blockwise(A.view(G * Mmax, K))
+    qa2 = torch.zeros_like(qa1)
+    sa2 = torch.ones_like(sa1)
+    for g in range(G):
+        if counts[g]:
+            q, s = binding.quantize_blockwise(A[g, :counts[g]])
+            qa2[g, :counts[g]] = q
+            sa2[g, :s.shape[0]] = s
     C1 = binding.grouped_gemm_masked(qa1, sa1, dev(qb), dev(sb), mm)
-    C2 = binding.grouped_gemm_masked(qa2.view(G, Mmax, K), sa2.view(G, Mmax // 128, -1), dev(qb), dev(sb), mm)
+    C2 = binding.grouped_gemm_masked(qa2, sa2, dev(qb), dev(sb), mm)
     torch.cuda.synchronize()
     assert binding.last_device_status() == 0
     for g in range(G):
