@@ -84,12 +84,13 @@ static_assert(128 * regs_producer<256>() + 256 * regs_epilogue<256>() <= kTileTh
                   128 * regs_producer<128>() + 256 * regs_epilogue<128>() <= kTileThreads * kRegsLaunch,
               "setmaxnreg split exceeds the registers the block is launched with");
 // Tiles run m-block-fastest through raster groups of kRasterM m-blocks x all n-tiles,
-// so a group's B tiles are read from L2 by its m-blocks.  Dense: 16 (measured 2.5 %
-// faster than 8 at 8192^3, the same at 4096^3); grouped: 8 (16 was about 1 % slower
-// on the 64-expert MoE GEMM).
+// so a group's B tiles are read from L2 by its m-blocks.  Dense: 32 (measured at
+// 8192^3: 432 us, against 437 with 16, 446-455 with 8 and 465 with 64; at 4096^3,
+// a single group, up to 3 % faster than 16); grouped: 8 (16 was about 1 % slower on
+// the 64-expert MoE GEMM).
 template <int GMODE>
 __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int &mb, int &nb) {
-    constexpr int kRasterM = GMODE == kDense ? 16 : 8;
+    constexpr int kRasterM = GMODE == kDense ? 32 : 8;
     const int group = t / (kRasterM * num_n);
     const int first_m = group * kRasterM;
     const int gm = min(kRasterM, num_m - first_m);
