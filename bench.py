@@ -70,19 +70,19 @@ SKINNY_GRAPH_STEPS = 240
 # since the capture reports null.
 NCU_TRAFFIC = {
     # tile_gemm_kernel<256,kDense,4,2,0>, dense 512^3 (16 half-tile units): 0.56 MB read + 0.00 MB written
-    ("dense_512", "gemm_tile.cu", "cef735b8d8ae9785"): 555520,
-    # tile_gemm_kernel<256,kDense,4,2,0>, dense 4096^3 (1% outlier rows): 33.59 MB read + 2.13 MB written
-    ("dense_4096_outliers", "gemm_tile.cu", "cef735b8d8ae9785"): 35721728,
-    # tile_gemm_kernel<256,kDense,4,2,0>, dense 8192^3: 232.78 MB read + 119.05 MB written
-    ("dense_8192", "gemm_tile.cu", "cef735b8d8ae9785"): 351839232,
-    # tile_gemm_kernel<256,kContiguous,4,2,0>, 8 experts N=K=4096: 208.55 MB read + 119.79 MB written
-    ("moe_g8", "gemm_tile.cu", "cef735b8d8ae9785"): 328337408,
-    # tile_gemm_kernel<256,kContiguous,4,2,0>, 64 experts N=2048 K=7168: 1380.04 MB read + 145.07 MB written
-    ("moe_g64_zipf", "gemm_tile.cu", "cef735b8d8ae9785"): 1525109760,
-    # tile_gemm_kernel<256,kDense,4,2,1> (one A scale per row and 128-K group), dense 4096^3: 34.13 MB read + 2.26 MB written
-    ("dense_4096_outliers_1x128", "gemm_tile.cu", "cef735b8d8ae9785"): 36381440,
-    # tile_gemm_kernel<256,kMasked,4,2,0>, 8 experts in 6912-row slabs, N=K=4096: 208.73 MB read + 115.58 MB written
-    ("moe_masked_g8", "gemm_tile.cu", "cef735b8d8ae9785"): 324316672,
+    ("dense_512", "gemm_tile.cu", "0fd177e660881d01"): 555264,
+    # tile_gemm_kernel<256,kDense,4,2,0>, dense 4096^3 (1% outlier rows): 33.59 MB read + 2.43 MB written
+    ("dense_4096_outliers", "gemm_tile.cu", "0fd177e660881d01"): 36018944,
+    # tile_gemm_kernel<256,kDense,4,2,0>, dense 8192^3: 223.69 MB read + 117.10 MB written
+    ("dense_8192", "gemm_tile.cu", "0fd177e660881d01"): 340789248,
+    # tile_gemm_kernel<256,kContiguous,4,2,0>, 8 experts N=K=4096: 210.28 MB read + 118.86 MB written
+    ("moe_g8", "gemm_tile.cu", "0fd177e660881d01"): 329131264,
+    # tile_gemm_kernel<256,kContiguous,4,2,0>, 64 experts N=2048 K=7168: 1404.68 MB read + 145.07 MB written
+    ("moe_g64_zipf", "gemm_tile.cu", "0fd177e660881d01"): 1549749504,
+    # tile_gemm_kernel<256,kDense,4,2,1> (one A scale per row and 128-K group), dense 4096^3: 34.11 MB read + 2.20 MB written
+    ("dense_4096_outliers_1x128", "gemm_tile.cu", "0fd177e660881d01"): 36318464,
+    # tile_gemm_kernel<256,kMasked,4,2,0>, 8 experts in 6912-row slabs, N=K=4096: 211.24 MB read + 114.73 MB written
+    ("moe_masked_g8", "gemm_tile.cu", "0fd177e660881d01"): 325969664,
     # skinny_gemm_kernel<16,8,8,0> M=1 and M=16; <64,8,8,0> M=64; <128,6,4,0> M=128; <16,8,8,1> the
     # one-launch fused M=1 (N=K=4096): B once, nothing written back to DRAM within the capture
     ("skinny_m1", "gemm_skinny.cu", "e7452d79db77bcd8"): 16813824,

@@ -437,11 +437,16 @@ __global__ void __launch_bounds__(kTileThreads, 1)
             ScaleStream scales;
             scales.start(ROWS ? nullptr : p.sA + static_cast<int64_t>(ti.sa_row) * Kb,
                          p.sB + static_cast<int64_t>(sb_row) * Kb, 0, n_valid ? Kb : 0);
-            // ROWS: this thread's row scales, loaded two K blocks ahead
+            // ROWS: this thread's row scales, loaded two K blocks ahead through a pointer that
+            // advances by M floats a K block (recomputing the 64-bit address each K block
+            // spilled registers and cost 15 %: 80.9 vs 68.5 us at 4096^3, measured)
             const int my_row = ti.a_row + quarter * 32 + lane;
             const bool row_ok = ROWS && my_row < p.M;
-            float sa_next = row_ok ? __ldg(p.sA + my_row) : 0.0f;
-            float sa_next2 = (row_ok && Kb > 1) ? __ldg(p.sA + p.M + my_row) : 0.0f;
+            const float *sa_ptr = p.sA + (row_ok ? my_row : 0);  // advances one K block (M floats) per load
+            float sa_next = row_ok ? __ldg(sa_ptr) : 0.0f;
+            sa_ptr += p.M;
+            float sa_next2 = (row_ok && Kb > 1) ? __ldg(sa_ptr) : 0.0f;
+            sa_ptr += p.M;
 #pragma unroll
             for (int i = 0; i < kColsPerWarp / 2; ++i) acc[i] = make_float2(0.0f, 0.0f);
             for (int kb = 0; kb < Kb; ++kb, ++kc) {
@@ -451,7 +456,8 @@ __global__ void __launch_bounds__(kTileThreads, 1)
                 if (ROWS) {
                     const float sa = sa_next;
                     sa_next = sa_next2;
-                    sa_next2 = (row_ok && kb + 2 < Kb) ? __ldg(p.sA + static_cast<int64_t>(kb + 2) * p.M + my_row) : 0.0f;
+                    sa_next2 = (row_ok && kb + 2 < Kb) ? __ldg(sa_ptr) : 0.0f;
+                    sa_ptr += p.M;
                     scale = sa * scale;  // fl32(sA[row][kb] * sB[n/128][kb])
                 }
                 const float2 s2 = make_float2(scale, scale);
