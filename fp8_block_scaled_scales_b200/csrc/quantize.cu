@@ -24,33 +24,17 @@
 namespace dg {
 
 constexpr int kQuantThreads = 256;
+// Masked layout: CTAs per slab and column block, each taking every kMaskedRowCtas-th
+// token-holding row block.  Measured on 8 x 6912-row slabs for 16384 tokens: 4 ->
+// 71 us, 8 -> 54, 16 -> 47-49, 24 -> 49, 32 -> 51; one CTA per block 66.
+constexpr int64_t kMaskedRowCtas = 16;
 
-// Four CTAs per SM (64 registers): measured 8 % faster than three on the 262 M-element
-// MoE activations (147.5 vs 160.1 us), the extra warps hiding load latency.
-// MASKED: X is slabs of R rows each; slab g holds masked_m[g] tokens (clamped to
-// [0, R]) in its first rows and is quantized as the matrix of those rows alone: the
-// last token block's amax covers its tokens only, rows past the count are neither
-// read nor written, and the blocks past the last token are skipped (their Q and S
-// are left as they are).  Block (g, lb, bc) is CTA (g * Rb + lb) * Cb + bc and
-// writes scale S[that index].  Otherwise one matrix of R rows.
-template <bool MASKED>
-__global__ void __launch_bounds__(kQuantThreads, 4)
-    quantize_kernel(const uint16_t *__restrict__ X, int64_t R, int64_t C, int64_t Cb, uint8_t *__restrict__ Q,
-                    float *__restrict__ S, const int32_t *__restrict__ masked_m, int64_t Rb) {
-    __shared__ uint32_t red[kQuantThreads / 32];
-    // The GEMM that follows may start its set-up (and its weight prefetch into L2)
-    // at once: it still waits for this grid to complete before reading Q and S.
-    // Measured 5 % shorter for a quantize + skinny GEMM step at M = 16.
-    grid_dep_launch_dependents();
-    grid_dep_wait();  // X (and masked_m) may come from the previous kernel
-    const int64_t blk = blockIdx.x;
-    const int64_t br = blk / Cb, bc = blk - br * Cb;
-    const int64_t g = MASKED ? br / Rb : 0, lb = MASKED ? br - g * Rb : br;  // slab, row block inside it
-    // rows of this matrix: the slab's tokens when masked
-    const int64_t rows = MASKED ? min(max(static_cast<int64_t>(__ldg(masked_m + g)), int64_t(0)), R) : R;
-    if (MASKED && lb * 128 >= rows) return;  // no token in this block
-    const uint16_t *Xs = X + g * R * C;
-    uint8_t *Qs = Q + g * R * C;
+// One 128x128 block: rows lb*128 .. of the matrix Xs (R rows in all, of which `rows`
+// hold data), column block bc; scale into *Sp.  red: one word per warp, unused by
+// this CTA since the barrier before its previous block.
+__device__ __forceinline__ void quantize_block(const uint16_t *__restrict__ Xs, uint8_t *__restrict__ Qs,
+                                               float *__restrict__ Sp, int64_t C, int64_t rows, int64_t lb,
+                                               int64_t bc, uint32_t *red) {
     const int tid = static_cast<int>(threadIdx.x);
     const int chunk = tid & 15;  // 8-element column group
     const int sub = tid >> 4;    // 0..15
@@ -81,14 +65,58 @@ __global__ void __launch_bounds__(kQuantThreads, 4)
 #pragma unroll
     for (int i = 1; i < kQuantThreads / 32; ++i) m = max(m, red[i]);
     const BlockScale bs = block_scale(m);
-    const float s = bs.s;
-    if (tid == 0) S[br * Cb + bc] = s;
+    if (tid == 0) *Sp = bs.s;
 
     uint8_t *qp = Qs + row0 * C + col;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         if (i >= nr) break;
         *reinterpret_cast<uint2 *>(qp + i * step) = quantize8(v[i], bs);
+    }
+}
+
+// One CTA per block; four CTAs per SM (64 registers): measured 8 % faster than three
+// on the 262 M-element MoE activations (147.5 vs 160.1 us), the extra warps hiding
+// load latency.
+__global__ void __launch_bounds__(kQuantThreads, 4)
+    quantize_kernel(const uint16_t *__restrict__ X, int64_t R, int64_t C, int64_t Cb, uint8_t *__restrict__ Q,
+                    float *__restrict__ S) {
+    __shared__ uint32_t red[kQuantThreads / 32];
+    // The GEMM that follows may start its set-up (and its weight prefetch into L2)
+    // at once: it still waits for this grid to complete before reading Q and S.
+    // Measured 5 % shorter for a quantize + skinny GEMM step at M = 16.
+    grid_dep_launch_dependents();
+    grid_dep_wait();  // X may come from the previous kernel
+    const int64_t blk = blockIdx.x;
+    const int64_t lb = blk / Cb, bc = blk - lb * Cb;
+    quantize_block(X, Q, S + blk, C, R, lb, bc, red);
+}
+
+// The masked MoE layout: X is G slabs of R rows each; slab g holds masked_m[g] tokens
+// (clamped to [0, R]) in its first rows and is quantized as the matrix of those rows
+// alone: the last token block's amax covers its tokens only, rows past the count are
+// neither read nor written, and the blocks past the last token are skipped (their Q
+// and S are left as they are).  Block (g, lb, bc) writes scale S[(g * Rb + lb) * Cb +
+// bc].  CTA (g, y, bc) takes the slab's row blocks y, y + Ry, ... that hold tokens, so
+// mostly empty slabs cost few CTAs (one CTA per block: 9700 of 13800 CTAs exited at
+// once on 8 x 6912-row slabs for 16384 tokens).
+__global__ void __launch_bounds__(kQuantThreads, 4)
+    quantize_masked_kernel(const uint16_t *__restrict__ X, int64_t R, int64_t C, int64_t Cb,
+                           uint8_t *__restrict__ Q, float *__restrict__ S, const int32_t *__restrict__ masked_m,
+                           int64_t Rb, int64_t Ry) {
+    __shared__ uint32_t red[2][kQuantThreads / 32];
+    grid_dep_launch_dependents();  // as in quantize_kernel
+    grid_dep_wait();               // X and masked_m may come from the previous kernel
+    const int64_t blk = blockIdx.x;
+    const int64_t gy = blk / Cb, bc = blk - gy * Cb;
+    const int64_t g = gy / Ry, y = gy - g * Ry;
+    const int64_t rows = min(max(static_cast<int64_t>(__ldg(masked_m + g)), int64_t(0)), R);
+    const uint16_t *Xs = X + g * R * C;
+    uint8_t *Qs = Q + g * R * C;
+    int par = 0;
+    for (int64_t lb = y; lb * 128 < rows; lb += Ry) {
+        quantize_block(Xs, Qs, S + (g * Rb + lb) * Cb + bc, C, rows, lb, bc, red[par]);
+        par ^= 1;
     }
 }
 
@@ -146,11 +174,14 @@ dg_status_t launch_quantize_masked(const void *X, int64_t slabs, int64_t rows, i
     const int64_t Rb = (rows + 127) / 128, Cb = (cols + 127) / 128;
     const int64_t blocks = slabs * Rb * Cb;
     if (blocks > 0x7FFFFFFFLL) return DG_ERR_SHAPE;
-    if (masked_m == nullptr && slabs != 1) return DG_ERR_INVALID_ARG;
-    return masked_m ? launch_pdl(quantize_kernel<true>, static_cast<int>(blocks), kQuantThreads, 0, stream,
-                                 static_cast<const uint16_t *>(X), rows, cols, Cb, Q, S, masked_m, Rb)
-                    : launch_pdl(quantize_kernel<false>, static_cast<int>(blocks), kQuantThreads, 0, stream,
-                                 static_cast<const uint16_t *>(X), rows, cols, Cb, Q, S, masked_m, Rb);
+    if (masked_m == nullptr) {
+        if (slabs != 1) return DG_ERR_INVALID_ARG;
+        return launch_pdl(quantize_kernel, static_cast<int>(blocks), kQuantThreads, 0, stream,
+                          static_cast<const uint16_t *>(X), rows, cols, Cb, Q, S);
+    }
+    const int64_t Ry = min(Rb, kMaskedRowCtas);
+    return launch_pdl(quantize_masked_kernel, static_cast<int>(slabs * Ry * Cb), kQuantThreads, 0, stream,
+                      static_cast<const uint16_t *>(X), rows, cols, Cb, Q, S, masked_m, Rb, Ry);
 }
 
 }  // namespace dg
