@@ -75,9 +75,9 @@ __device__ __forceinline__ void quantize_block(const uint16_t *__restrict__ Xs, 
     }
 }
 
-// One CTA per block; four CTAs per SM (64 registers): measured 8 % faster than three
-// on the 262 M-element MoE activations (147.5 vs 160.1 us), the extra warps hiding
-// load latency.
+// One CTA per block; four CTAs per SM (at most 64 registers): measured 8 % faster
+// than three on the 262 M-element MoE activations (147.5 vs 160.1 us), the extra warps
+// hiding load latency.
 __global__ void __launch_bounds__(kQuantThreads, 4)
     quantize_kernel(const uint16_t *__restrict__ X, int64_t R, int64_t C, int64_t Cb, uint8_t *__restrict__ Q,
                     float *__restrict__ S) {
