@@ -130,6 +130,7 @@ def test_masked_largest_expert_count():
     (4, 200, 256, [0, 200, 77, 129]),        # an empty slab, a full one, partial last blocks
     (3, 384, 4000, [384, 1, 128]),           # K tail; a block boundary exactly at the count
     (2, 130, 144, [-5, 1000]),               # counts clamped to [0, M_max]
+    (2, 5120, 256, [5000, 2100]),            # 40 row blocks: each CTA of a slab takes several in turn
 ])
 def test_masked_quantizer_quantizes_each_slabs_tokens_alone(G, Mmax, K, counts):
     """Slab g's first counts[g] rows get, bit for bit, the block quantizer's codes and
