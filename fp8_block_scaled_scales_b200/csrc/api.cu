@@ -159,7 +159,7 @@ using namespace dg;
 
 extern "C" {
 
-int dg_version(void) { return 104; }
+int dg_version(void) { return 105; }
 
 const char *dg_status_string(dg_status_t s) {
     switch (s) {

@@ -296,7 +296,9 @@ dg_status_t dg_get_last_device_status(cudaStream_t stream);
 /* Library ABI version (major * 100 + minor).  1.01 added the BF16-activation,
  * per-token-scale and masked-MoE calls; 1.02 added DG_ERR_GROUP_OFFSETS; 1.03
  * added dg_fp8_gemm_blockscaled_bf16a_select and DG_KERNEL_SKINNY_FUSED; 1.04 added
- * dg_quantize_blockwise_masked.  Every 1.00 call is unchanged. */
+ * dg_quantize_blockwise_masked; 1.05: dg_quantize_blockwise_masked quantizes each
+ * expert's tokens as a matrix of their own (rows past the count no longer enter the
+ * last token block's amax).  Every 1.00 call is unchanged. */
 int dg_version(void);
 
 /*

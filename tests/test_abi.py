@@ -38,7 +38,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.dg_version() == 104
+    assert lib.dg_version() == 105
     for code, name in binding.STATUS_NAMES.items():
         assert lib.dg_status_string(code).decode().startswith(name)
     # the device-side group_offsets check has its own code, named in the header
