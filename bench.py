@@ -399,6 +399,15 @@ def aggregate_rate(world: int, units_per_rank_step: float, ms_per_step_max: floa
     return world * units_per_rank_step / (ms_per_step_max * 1e-3)
 
 
+def io_rows(w, rows_a: int):
+    """(first row, rows) of A and C that carry a step's data: of a masked slab its
+    tokens only (no result depends on the rows past a count), else all rows."""
+    from fp8_block_scaled_scales_b200.inputs import Masked
+    if isinstance(w, Masked):
+        return [(g * w.M_max, int(min(max(w.counts[g], 0), w.M_max))) for g in range(w.G) if w.counts[g] > 0]
+    return [(0, rows_a)]
+
+
 # --------------------------------------------------------------- device plans
 class Plan:
     """One workload on the device: inputs, the step's kernels, and its facts."""
@@ -419,9 +428,7 @@ class Plan:
         self.kernel_file = kernel_file_of(name)
         self.A_host = w.A.contiguous().reshape(rows_a, w.K)  # masked: the [G][M_max] slabs as rows
         self.A = self.A_host.to(dev)
-        # (first row, rows) of A and C that carry the step's data: a masked slab's tokens only
-        self.io_rows = ([(g * w.M_max, int(w.counts[g])) for g in range(w.G) if w.counts[g]] if self.masked
-                        else [(0, rows_a)])
+        self.io_rows = io_rows(w, rows_a)
         B = w.B.reshape(-1, w.K).to(dev) if (self.grouped or self.masked) else w.B.to(dev)
         self.qb, self.sb = binding.quantize_blockwise(B)  # cached weights
         del B

@@ -60,3 +60,11 @@ def test_grouped_and_masked_count_real_tokens(bench):
 def test_whole_job_rate_is_replicas_over_slowest(bench):
     assert bench.aggregate_rate(1, 1e12, 1.0) == pytest.approx(1e15)
     assert bench.aggregate_rate(8, 1e12, 2.0) == pytest.approx(8e12 / 2e-3)
+
+
+def test_e2e_copies_a_masked_slabs_tokens_only(bench):
+    from fp8_block_scaled_scales_b200 import inputs
+    m = inputs.Masked("m", 3, 512, 256, 256, np.array([130, 0, 512]), None, None, 0)
+    assert bench.io_rows(m, 3 * 512) == [(0, 130), (1024, 512)]
+    d = inputs.Dense("d", 300, 256, 256, None, None, 0, np.zeros(0, np.int64))
+    assert bench.io_rows(d, 300) == [(0, 300)]
