@@ -167,6 +167,12 @@ def _every_tile_check(d, kernel="auto", seed=0):
     return check(c[rows], ref, rms, d.name)
 
 
+def test_dense_past_one_raster_group():
+    """36 m-blocks: a whole raster group of 32 m-blocks, then a partial one of 4, and a
+    ragged last block; every tile compared."""
+    _every_tile_check(inputs.dense_custom(4500, 768, 384, seed=8800))
+
+
 def test_dense_4096_outliers_workload():
     """The headline workload compared in full: all 4096 x 4096 outputs."""
     d = inputs.dense_4096_outliers()
